@@ -1,0 +1,146 @@
+/*
+ * mla_b200.h — C ABI of the B200 (sm_100a) MLA paged-KV decode library.
+ *
+ * Operation (cnblogs "DeepSeek 开源记-第1天-FlashMLA", §2 核心功能 and §6.2
+ * 基本使用): Multi-head Latent Attention decoding over a paged BF16 latent
+ * KV cache.  Every cached token holds one row of d = 576 values per KV head
+ * (512 latent + 64 rotary); the value vector is the first dv = 512 values of
+ * the same row; pages hold 64 tokens (m.ygpos.cn "DeepSeek代碼開源第一彈Flash
+ * MLA", release list) and are addressed through a block table; sequences have
+ * variable lengths.  For every query row:
+ *     x_j = scale * <q, K_j>,  lse = ln sum_j exp(x_j),
+ *     O   = sum_j exp(x_j - lse) * V_j.
+ *
+ * Conventions for every call below
+ *   - Pointers named *_d are device pointers; all are owned by the caller and
+ *     must stay valid until the stream work completes.  The library allocates
+ *     no device memory and never synchronises the stream.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream).
+ *   - Return value: MLA_OK or a negative MLA_ERR_* code; on error nothing is
+ *     launched.  Errors detected on the device (bad page ids, sequence longer
+ *     than its block-table row, a bounded wait that ran out) are written to
+ *     the optional `status_d` word (int32, 0 = OK) and the affected rows are
+ *     zeroed; read it after synchronising.
+ *   - Layouts are dense, row-major, contiguous (innermost index last).
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_OK                0
+#define MLA_ERR_INVALID_ARG  -1   /* null pointer, bad alignment, bad sizes      */
+#define MLA_ERR_UNSUPPORTED  -2   /* d != 576, dv != 512, device not sm_100       */
+#define MLA_ERR_WORKSPACE    -3   /* workspace missing or too small              */
+#define MLA_ERR_CUDA         -4   /* a CUDA runtime/driver call failed           */
+#define MLA_ERR_TIMEOUT      -5   /* device-side bounded wait gave up (status_d) */
+#define MLA_ERR_BAD_INPUT    -6   /* device-side input check failed (status_d)   */
+
+#define MLA_HEAD_DIM   576
+#define MLA_VALUE_DIM  512
+#define MLA_PAGE_SIZE  64
+#define MLA_MD_WORDS   8      /* int32 words per tile-scheduler entry */
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* mla_status_string(int status);
+
+/* Number of SMs of the current device (cached per device), or a negative
+ * MLA_ERR_* code. */
+int mla_device_sm_count(void);
+
+/* Rows per decode CTA for `rows_per_kv` query rows per KV head: 16, 32 or 64.
+ * Host-only, pure. */
+int mla_rows_per_block(int rows_per_kv);
+
+/* Number G of scheduler parts ("tile_scheduler_metadata" entries) for the
+ * given shape: max(1, num_sms / (h_kv * ceil(rows_per_kv / rows_per_block))).
+ * Host-only, pure.  Returns a negative MLA_ERR_* code on bad arguments. */
+int mla_num_parts(int rows_per_kv, int h_kv, int num_sms);
+
+/*
+ * Tile-scheduler metadata (jsxs2.com "什麼是FlashMLA", §3.1 分塊調度與並行
+ * 計算: the work is cut into blocks and scheduled over the SMs; cnblogs §6.2:
+ * get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) returns
+ * tile_scheduler_metadata and num_splits).
+ *
+ *   cache_seqlens_d  int32[batch]            sequence lengths L_b >= 0
+ *   rows_per_kv      s_q * h_q / h_kv
+ *   h_kv             number of KV heads
+ *   num_sms          SMs to schedule over (<= 0: this device's SM count)
+ *   tile_md_d        int32[G * MLA_MD_WORDS]  out: per part
+ *                    (begin_b, begin_page, end_b, end_page, first_piece,
+ *                     n_pieces, 0, 0), end exclusive
+ *   num_splits_d     int32[batch + 1]        out: prefix sum of pieces per
+ *                    sequence
+ *   num_parts_out    host int*, out: G (may be NULL)
+ * One single-CTA kernel; integer arithmetic only (bit-exact, deterministic).
+ */
+int mla_get_metadata(const int32_t* cache_seqlens_d, int batch, int rows_per_kv, int h_kv,
+                     int num_sms, int32_t* tile_md_d, int32_t* num_splits_d,
+                     int* num_parts_out, void* stream);
+
+/* Bytes of device workspace mla_decode_paged needs for split partials:
+ * (batch + num_parts) * h_kv * rows_per_kv * (dv + 1) * 4, rounded up to
+ * 256.  Returns 0 on bad arguments. */
+size_t mla_workspace_bytes(int batch, int rows_per_kv, int h_kv, int dv, int num_parts);
+
+/*
+ * Split-KV MLA decode (cnblogs §6.2: flash_mla_with_kvcache(q, blocked_k,
+ * block_table, cache_seqlens, dv, tile_scheduler_metadata, num_splits,
+ * causal) -> output, lse; compute flow cnblogs §4.1: load, blockwise scores,
+ * softmax, merge of the outputs).
+ *
+ *   q_d             bf16 [batch, s_q, h_q, d]             (16-byte aligned)
+ *   k_cache_d       bf16 [num_pages, 64, h_kv, d]          (16-byte aligned)
+ *   block_table_d   int32 [batch, max_pages_per_seq]; entries for pages at
+ *                   or beyond ceil(L_b/64) are never read
+ *   cache_seqlens_d int32 [batch]; L_b <= 64 * max_pages_per_seq required
+ *   d, dv           must be 576 and 512
+ *   tile_md_d, num_splits_d, num_parts: exactly as produced by
+ *                   mla_get_metadata for the same seqlens, rows_per_kv, h_kv
+ *   causal          0/1; query token s sees keys j < L - (s_q - 1 - s)
+ *   softmax_scale   multiplies <q, K_j>; pass 576^-0.5 for the usual scale
+ *   workspace_d     >= mla_workspace_bytes(...) bytes, 256-byte aligned
+ *   out_d           bf16 [batch, s_q, h_q, dv]             (16-byte aligned)
+ *   lse_d           fp32 [batch, s_q, h_q]; natural log; -inf for rows that
+ *                   see no key (their out row is 0)
+ *   status_d        optional int32 device word (see conventions)
+ * Launches the decode kernel and, if any sequence is split or empty, the
+ * combine kernel, both on `stream`.
+ */
+int mla_decode_paged(const void* q_d, const void* k_cache_d, int num_pages,
+                     const int32_t* block_table_d, int max_pages_per_seq,
+                     const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
+                     int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d,
+                     int num_parts, int causal, float softmax_scale,
+                     void* workspace_d, size_t workspace_bytes,
+                     void* out_d, float* lse_d, int32_t* status_d, void* stream);
+
+/*
+ * Debug/testing variant of mla_decode_paged with extra knobs; same contract
+ * otherwise.
+ *   debug_flags  bit 0: the softmax warps wait on a barrier that nothing
+ *                signals, so the bounded wait must run out and report
+ *                MLA_ERR_TIMEOUT through status_d (fault detection test).
+ *   timeout_ns   limit of every device-side wait (0 = default, 4 s).
+ */
+int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,
+                        const int32_t* block_table_d, int max_pages_per_seq,
+                        const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
+                        int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d,
+                        int num_parts, int causal, float softmax_scale,
+                        void* workspace_d, size_t workspace_bytes,
+                        void* out_d, float* lse_d, int32_t* status_d,
+                        int debug_flags, unsigned long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,94 @@
+// combine.cu — merge of split-KV partial results (cnblogs "DeepSeek 开源记-第1天-
+// FlashMLA", §4.1 计算流程: 输出结果合并).
+//
+// For a row whose sequence was cut into n >= 2 pieces, each piece i left
+// (O_i, lse_i) with O_i already normalised by its own denominator.  Then
+//     lse = ln sum_i exp(lse_i),   O = sum_i exp(lse_i - lse) * O_i.
+// Pieces with lse_i = -inf weigh nothing; if all are -inf the row is O = 0,
+// lse = -inf.  Sequences with no piece (empty) get the same zero row.
+// Sequences with exactly one piece were written by the decode kernel and are
+// skipped here.
+//
+// One warp per query row: each lane owns 16 of the 512 values, reads them with
+// 16-byte loads per piece and writes 16 bf16 (two 16-byte stores), so a warp
+// moves whole 2 KB partial rows and a 1 KB output row.
+#include "decode.cuh"
+
+namespace mla {
+
+namespace {
+
+constexpr int kRowsPerBlock = 4;
+
+__global__ void __launch_bounds__(32 * kRowsPerBlock)
+mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restrict__ o_part,
+                   const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ out,
+                   float* __restrict__ lse, int batch, int s_q, int h_q, int h_kv, int R) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRowsPerBlock + warp;
+  const int g = blockIdx.y, b = blockIdx.z;
+  if (r >= R) return;
+  const int first = __ldg(num_splits + b);
+  const int n = __ldg(num_splits + b + 1) - first;
+  if (n == 1) return;
+
+  const int hg = h_q / h_kv;
+  const int srow = r / hg, h = g * hg + r % hg;
+  const size_t out_row = (static_cast<size_t>(b) * s_q + srow) * h_q + h;
+
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  float top = -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    top = fmaxf(top, __ldg(lse_part + (static_cast<size_t>(first + i) * h_kv + g) * R + r));
+  }
+  float total_lse = -INFINITY;
+  if (top != -INFINITY) {
+    float wsum = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const size_t row = (static_cast<size_t>(first + i) * h_kv + g) * R + r;
+      const float li = __ldg(lse_part + row);
+      const float w = li == -INFINITY ? 0.f : expf(li - top);
+      wsum += w;
+      if (w != 0.f) {
+        const float4* src = reinterpret_cast<const float4*>(o_part + row * 512) + lane * 4;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 x = __ldg(src + v);
+          acc[4 * v + 0] += w * x.x;
+          acc[4 * v + 1] += w * x.y;
+          acc[4 * v + 2] += w * x.z;
+          acc[4 * v + 3] += w * x.w;
+        }
+      }
+    }
+    const float inv = 1.f / wsum;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] *= inv;
+    total_lse = top + logf(wsum);
+  }
+  uint32_t packed[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    packed[i] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + out_row * 512) + lane * 2;
+  dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  if (lane == 0) lse[out_row] = total_lse;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
+                           __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
+                           cudaStream_t stream) {
+  const dim3 grid((R + kRowsPerBlock - 1) / kRowsPerBlock, h_kv, batch);
+  mla_combine_kernel<<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, out, lse, batch,
+                                                              s_q, h_q, h_kv, R);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

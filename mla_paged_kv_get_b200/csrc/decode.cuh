@@ -1,0 +1,40 @@
+// decode.cuh — launch interface of the decode, combine and metadata kernels
+// (host side of the C ABI in capi.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+struct DecodeArgs {
+  const int32_t* block_table;   // [batch, max_pages]
+  const int32_t* seqlens;       // [batch]
+  const int32_t* tile_md;       // [num_parts, 8]
+  const int32_t* num_splits;    // [batch + 1]
+  __nv_bfloat16* out;           // [batch, s_q, h_q, 512]
+  float* lse;                   // [batch, s_q, h_q]
+  float* o_part;                // [max_pieces, h_kv, R, 512]
+  float* lse_part;              // [max_pieces, h_kv, R]
+  int32_t* status;              // optional
+  int batch, s_q, h_q, h_kv, hg, R;
+  int max_pages, num_pages, causal, num_parts, max_pieces;
+  float scale_log2;             // softmax_scale * log2(e)
+  int debug_flags;
+  unsigned long long timeout_ns;
+};
+
+int decode_smem_bytes(int rows_per_block);
+cudaError_t launch_decode(int rows_per_block, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+                          const DecodeArgs& a, int row_blocks, cudaStream_t stream);
+
+cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
+                           __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
+                           cudaStream_t stream);
+
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,
+                            int32_t* num_splits, cudaStream_t stream);
+
+}  // namespace mla

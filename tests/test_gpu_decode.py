@@ -1,0 +1,189 @@
+"""GPU parity: metadata bit-exact, decode within the stated tolerances, through the C ABI."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from mla_paged_kv_get_b200 import binding, inputs
+from oracle import mla_oracle as mo
+from oracle import schedule as sch
+
+from gpu_util import compare, to_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    binding.load_library()
+
+
+def run_gpu(w, num_sms=None, **kw):
+    q, k, bt, sl = to_gpu(w)
+    tile_md, num_splits = binding.get_metadata(sl, w.rows_per_kv, w.h_kv, num_sms)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = binding.decode_paged(q, k, bt, sl, 512, tile_md, num_splits, causal=w.causal,
+                                    softmax_scale=w.scale, status=status, **kw)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, binding.status_string(int(status.item()))
+    return out, lse, tile_md, num_splits
+
+
+def oracle(w, batches=None):
+    return mo.decode_dense(w.q, w.k_cache, w.block_table, w.seqlens, w.h_kv, w.causal, w.scale,
+                           batches=batches)
+
+
+# ---------------------------------------------------------------- metadata
+
+@pytest.mark.parametrize("seed", range(12))
+def test_metadata_bit_exact(seed):
+    g = torch.Generator().manual_seed(seed)
+    B = [1, 2, 7, 64, 128, 132, 300, 1000][seed % 8]
+    mode = seed % 4
+    if mode == 0:
+        lens = torch.randint(0, 8193, (B,), generator=g)
+    elif mode == 1:
+        lens = torch.tensor([[0, 1, 63, 64, 65, 127, 128][i % 7] for i in range(B)])
+    elif mode == 2:
+        lens = torch.randint(32768, 65537, (B,), generator=g)
+    else:
+        lens = torch.full((B,), 4096)
+    for rows, h_kv, sms in [(16, 1, 148), (128, 1, 148), (128, 1, 7), (32, 2, 148), (16, 1, 1), (256, 1, 148)]:
+        md, ns = binding.get_metadata(lens.to(torch.int32).cuda(), rows, h_kv, sms)
+        md_ref, ns_ref = sch.get_metadata(lens.tolist(), rows, h_kv, sms)
+        assert md.cpu().tolist() == md_ref
+        assert ns.cpu().tolist() == ns_ref
+
+
+# ---------------------------------------------------------------- decode parity
+
+def test_tiny_config():
+    w = inputs.config(1)
+    out, lse, _, _ = run_gpu(w)
+    o_ref, l_ref = oracle(w)
+    compare(w, out, lse, o_ref, l_ref, what="tiny")
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_small_cases(seed):
+    w = inputs.random_case(100 + seed, max_batch=5, max_len=700, h_q_choices=(16, 32, 64, 128),
+                           s_q_choices=(1, 2), h_kv_choices=(1, 2) if seed % 3 == 0 else (1,))
+    sms = [148, 7, 3, 1][seed % 4]
+    out, lse, _, _ = run_gpu(w, num_sms=sms)
+    o_ref, l_ref = oracle(w)
+    compare(w, out, lse, o_ref, l_ref, what=f"random {seed}")
+
+
+@pytest.mark.parametrize("rows", [(1, 16), (1, 32), (2, 16), (1, 64), (1, 128), (2, 64), (4, 32), (1, 8), (3, 16)])
+def test_row_shapes(rows):
+    s_q, h_q = rows
+    w = inputs.build(f"rows{s_q}x{h_q}", [1, 63, 64, 65, 129, 300], s_q=s_q, h_q=h_q, causal=s_q > 1, seed=77)
+    out, lse, _, _ = run_gpu(w, num_sms=5)
+    o_ref, l_ref = oracle(w)
+    compare(w, out, lse, o_ref, l_ref, what=f"s_q={s_q} h_q={h_q}")
+
+
+def test_edge_lengths_and_empty_rows():
+    # empty sequence, single token, exact page, page + 1, causal rows that see nothing
+    w = inputs.build("edges", [0, 1, 64, 65, 2, 128], s_q=2, h_q=16, causal=True, seed=5)
+    out, lse, _, ns = run_gpu(w, num_sms=4)
+    o_ref, l_ref = oracle(w)
+    compare(w, out, lse, o_ref, l_ref, what="edges")
+    o = out.float().cpu()
+    assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0].cpu()))
+    # seqlen 1, causal s_q=2: token 0 sees nothing, token 1 sees key 0 -> O = V_0
+    assert torch.all(o[1, 0] == 0)
+    v0 = w.k_cache[w.block_table[1, 0], 0, 0, :512].float()
+    assert (o[1, 1] - v0).abs().max() <= 2 ** -8 * v0.abs().max()
+
+
+def test_page_permutation_bit_identical():
+    w = inputs.build("perm", [700, 333, 64], s_q=1, h_q=128, seed=6)
+    out0, lse0, _, _ = run_gpu(w)
+    perm = torch.randperm(w.k_cache.shape[0], generator=torch.Generator().manual_seed(1))
+    k2 = torch.empty_like(w.k_cache)
+    k2[perm] = w.k_cache
+    w.k_cache = k2
+    w.block_table = perm[w.block_table.long()].to(torch.int32)
+    out1, lse1, _, _ = run_gpu(w)
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
+
+
+def test_poison_does_not_leak():
+    w = inputs.build("poison", [100, 64, 129], s_q=2, h_q=16, causal=True, seed=8)
+    out0, lse0, _, _ = run_gpu(w, num_sms=3)
+    w2 = inputs.build("poison", [100, 64, 129], s_q=2, h_q=16, causal=True, seed=8, poison=-7.5)
+    out1, lse1, _, _ = run_gpu(w2, num_sms=3)
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
+
+
+def test_forced_part_counts_agree():
+    w = inputs.build("parts", [5000, 3000, 64, 1], s_q=1, h_q=128, seed=9)
+    o_ref, l_ref = oracle(w)
+    for sms in (1, 2, 9, 148):
+        out, lse, _, _ = run_gpu(w, num_sms=sms)
+        compare(w, out, lse, o_ref, l_ref, what=f"num_sms={sms}")
+
+
+@pytest.mark.parametrize("index", [2, 3, 4, 5])
+def test_full_size_configs_sampled(index):
+    """The full workloads in the launch configuration the bench uses; the oracle
+    checks a sample of sequences (first, last and a spread in between)."""
+    w = inputs.config(index)
+    out, lse, md, ns = run_gpu(w)
+    B = w.batch
+    sample = sorted(set([0, B - 1] + list(range(1, B - 1, max(1, B // 6)))))[:8]
+    o_ref, l_ref = oracle(w, batches=sample)
+    compare(w, out, lse, o_ref, l_ref, batches=sample, what=f"config {index}")
+    # metadata of the full workload is bit-exact as well
+    md_ref, ns_ref = sch.get_metadata(w.seqlens.tolist(), w.rows_per_kv, w.h_kv, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert md.cpu().tolist() == md_ref and ns.cpu().tolist() == ns_ref
+    # every row is finite and every lse finite (all sequences are non-empty)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+# ---------------------------------------------------------------- failure paths
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    w = inputs.config(1)
+    q, k, bt, sl = to_gpu(w)
+    md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, status=status,
+                         debug_flags=1, timeout_ns=20_000_000)
+    torch.cuda.synchronize()
+    assert int(status.item()) == binding.MLA_ERR_TIMEOUT
+    out, lse, _, _ = run_gpu(w)           # the context is still usable
+    o_ref, l_ref = oracle(w)
+    compare(w, out, lse, o_ref, l_ref, what="after timeout")
+
+
+def test_corrupt_page_id_is_reported_not_read():
+    w = inputs.build("corrupt", [200, 100], s_q=1, h_q=16, seed=10)
+    w.block_table[0, 1] = 10 ** 6          # beyond the cache
+    q, k, bt, sl = to_gpu(w)
+    md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == binding.MLA_ERR_BAD_INPUT
+    o_ref, l_ref = oracle(w, batches=[1])  # the untouched sequence is still right
+    compare(w, out, lse, o_ref, l_ref, batches=[1], what="corrupt")
+
+
+def test_host_side_argument_errors():
+    w = inputs.config(1)
+    q, k, bt, sl = to_gpu(w)
+    md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv)
+    with pytest.raises(binding.MLAError):     # dv must be 512
+        binding.decode_paged(q, k, bt, sl, 256, md, ns)
+    with pytest.raises(binding.MLAError):     # workspace too small
+        binding.decode_paged(q, k, bt, sl, 512, md, ns,
+                             workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ValueError):           # wrong dtype is caught before the library
+        binding.decode_paged(q.float(), k, bt, sl, 512, md, ns)
