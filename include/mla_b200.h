@@ -128,6 +128,9 @@ int mla_decode_paged(const void* q_d, const void* k_cache_d, int num_pages,
  *   debug_flags  bit 0: the softmax warps wait on a barrier that nothing
  *                signals, so the bounded wait must run out and report
  *                MLA_ERR_TIMEOUT through status_d (fault detection test).
+ *                bit 1: launch only the decode kernel; the caller then calls
+ *                mla_combine with the same workspace (used to time the two
+ *                kernels separately).
  *   timeout_ns   limit of every device-side wait (0 = default, 4 s).
  */
 int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,
@@ -138,6 +141,17 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,
                         void* workspace_d, size_t workspace_bytes,
                         void* out_d, float* lse_d, int32_t* status_d,
                         int debug_flags, unsigned long long timeout_ns, void* stream);
+
+/*
+ * Merge of split partials (cnblogs §4.1 计算流程, 输出结果合并): for every query
+ * row of a sequence cut into n >= 2 pieces, lse = ln sum_i exp(lse_i) and
+ * O = sum_i exp(lse_i - lse) * O_i; sequences with no piece get O = 0 and
+ * lse = -inf; sequences with one piece are left untouched (the decode kernel
+ * wrote them).  workspace_d holds the partials mla_decode_paged_ex left with
+ * debug_flags bit 1; the other arguments are those of that call.
+ */
+int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch,
+                int s_q, int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream);
 
 #ifdef __cplusplus
 }

@@ -73,6 +73,8 @@ def load_library() -> ctypes.CDLL:
     lib.mla_decode_paged.restype = ci
     lib.mla_decode_paged_ex.argtypes = dec + [ci, ctypes.c_ulonglong, vp]
     lib.mla_decode_paged_ex.restype = ci
+    lib.mla_combine.argtypes = [i32p, vp, csz, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.mla_combine.restype = ci
     _lib = lib
     return lib
 

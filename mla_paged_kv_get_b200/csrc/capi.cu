@@ -220,8 +220,27 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int row_blocks = (R + n - 1) / n;
   if (mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (debug_flags & 2) return MLA_OK;
   if (mla::launch_combine(num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=
       cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch, int s_q,
+                int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream) {
+  if (num_splits_d == nullptr || workspace_d == nullptr || out_d == nullptr || lse_d == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65535 || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || num_parts < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(out_d, 16) || !aligned(workspace_d, 256)) return MLA_ERR_INVALID_ARG;
+  const int R = static_cast<int>(static_cast<long long>(s_q) * h_q / h_kv);
+  if (workspace_bytes < mla_workspace_bytes(batch, R, h_kv, MLA_VALUE_DIM, num_parts)) return MLA_ERR_WORKSPACE;
+  const size_t max_pieces = static_cast<size_t>(batch) + num_parts;
+  const float* o_part = static_cast<const float*>(workspace_d);
+  const float* lse_part = o_part + max_pieces * h_kv * R * MLA_VALUE_DIM;
+  if (mla::launch_combine(num_splits_d, o_part, lse_part, static_cast<__nv_bfloat16*>(out_d), lse_d, batch, s_q,
+                          h_q, h_kv, R, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
