@@ -153,6 +153,39 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,
 int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch,
                 int s_q, int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream);
 
+/*
+ * Allocation-free variant of mla_decode_paged.  The pages describe no such
+ * call; it has no counterpart there and exists for callers that cannot call
+ * cudaMalloc: code that runs where the device allocator belongs to someone
+ * else (a plugin or custom operator inside a host framework with its own
+ * memory pool), where allocation after start-up is forbidden by a fixed
+ * memory budget, or where the caller simply has no handle to allocate with.
+ *
+ * Same arguments and results as mla_decode_paged, minus the workspace: the
+ * split partials go to a scratch array of MLA_NOALLOC_SCRATCH_BYTES that the
+ * library holds in a file-scope __device__ variable, so every GPU that loads
+ * the library keeps those bytes until the process exits.  Nothing is
+ * allocated by this call (no cudaMalloc, cudaFree or allocating library
+ * routine).
+ *   - Returns MLA_ERR_WORKSPACE if the shape needs more than
+ *     MLA_NOALLOC_SCRATCH_BYTES (mla_workspace_bytes(...) larger than it).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call outside any stream capture.
+ *   - All calls share the one scratch array and it keeps the previous call's
+ *     contents; nothing in it needs to start at zero (every partial is written
+ *     before it is read).  Calls that overlap on the GPU (other streams, other
+ *     host threads) race on it: serialise them.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+int mla_decode_paged_noalloc(const void* q_d, const void* k_cache_d, int num_pages,
+                             const int32_t* block_table_d, int max_pages_per_seq,
+                             const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
+                             int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d,
+                             int num_parts, int causal, float softmax_scale,
+                             void* out_d, float* lse_d, int32_t* status_d, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
