@@ -80,6 +80,7 @@ int mla_num_parts(int rows_per_kv, int h_kv, int num_sms);
  *                    sequence
  *   num_parts_out    host int*, out: G (may be NULL)
  * One single-CTA kernel; integer arithmetic only (bit-exact, deterministic).
+ * Limits: batch <= 8192 and G <= 4096 (MLA_ERR_INVALID_ARG otherwise).
  */
 int mla_get_metadata(const int32_t* cache_seqlens_d, int batch, int rows_per_kv, int h_kv,
                      int num_sms, int32_t* tile_md_d, int32_t* num_splits_d,
@@ -131,6 +132,9 @@ int mla_decode_paged(const void* q_d, const void* k_cache_d, int num_pages,
  *                bit 1: launch only the decode kernel; the caller then calls
  *                mla_combine with the same workspace (used to time the two
  *                kernels separately).
+ *                bit 2: for more than 64 rows per KV head, use one CTA per
+ *                64-row block instead of CTA pairs (cross-check of the two
+ *                decode kernels).
  *   timeout_ns   limit of every device-side wait (0 = default, 4 s).
  */
 int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,

@@ -13,7 +13,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["capi.cu", "metadata.cu", "decode.cu", "combine.cu", "noalloc.cu"]
+SOURCES = ["capi.cu", "metadata.cu", "decode.cu", "decode_pair.cu", "combine.cu", "noalloc.cu"]
 LIB = os.path.join(HERE, "libmla_b200.so")
 
 

@@ -11,6 +11,7 @@
 
 namespace mla {
 int metadata_max_batch();
+int metadata_max_parts();
 }
 
 namespace {
@@ -112,7 +113,7 @@ int mla_get_metadata(const int32_t* cache_seqlens_d, int batch, int rows_per_kv,
     num_sms = d.sms;
   }
   const int g = mla_num_parts(rows_per_kv, h_kv, num_sms);
-  if (g < 1) return MLA_ERR_INVALID_ARG;
+  if (g < 1 || g > mla::metadata_max_parts()) return MLA_ERR_INVALID_ARG;
   if (mla::launch_metadata(cache_seqlens_d, batch, g, tile_md_d, num_splits_d,
                            static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
@@ -192,6 +193,7 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   }
 
   mla::DecodeArgs a;
+  a.k_cache = static_cast<const uint8_t*>(k_cache_d);
   a.block_table = block_table_d;
   a.seqlens = cache_seqlens_d;
   a.tile_md = tile_md_d;
@@ -219,7 +221,11 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int row_blocks = (R + n - 1) / n;
-  if (mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s) != cudaSuccess) return MLA_ERR_CUDA;
+  // 65..128+ rows per KV head: CTA pairs with 2-SM MMAs; otherwise one CTA per row block
+  const bool use_pair = R > 64 && !(debug_flags & 4);
+  const cudaError_t le = use_pair ? mla::launch_decode_pair(tm_k, tm_q, a, row_blocks, s)
+                                  : mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s);
+  if (le != cudaSuccess) return MLA_ERR_CUDA;
   if (debug_flags & 2) return MLA_OK;
   if (mla::launch_combine(num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=
       cudaSuccess)

@@ -38,13 +38,14 @@
 
 #include "ptx.cuh"
 #include "decode.cuh"
+#include "segments.cuh"
 
 namespace mla {
 
 namespace {
 
 constexpr int kKeys = 128;          // keys per tile (two pages)
-constexpr int kSlotBytes = 32768;   // one ring slot
+constexpr int kSlotBytes = 16384;   // one ring slot: two 64 x 64 boxes
 constexpr int kBoxBytes = 8192;     // one TMA box: 64 tokens x 64 bf16 columns
 constexpr int kThreads = 192;
 constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
@@ -53,13 +54,14 @@ constexpr int kSoftmaxBar = 1;      // named barrier of warps 0-3
 
 template <int N>
 struct Cfg {
-  static constexpr int kSlots = N == 64 ? 3 : (N == 32 ? 5 : 6);
+  static constexpr int kSlots = N == 64 ? 8 : (N == 32 ? 10 : 12);
+  static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
   static constexpr int kQBytes = N * 128 * 9;          // 9 chunks of [N rows][64 cols]
   static constexpr int kPBytes = kKeys * N * 2;        // P^T: [128 keys][N rows] bf16
   static constexpr int kTmemCols = N == 64 ? 512 : (N == 32 ? 256 : 128);
   static constexpr int kOffQ = kSlots * kSlotBytes;
   static constexpr int kOffP = kOffQ + kQBytes;
-  static constexpr int kOffCtrl = kOffP + 2 * kPBytes;
+  static constexpr int kOffCtrl = kOffP + kPBuf * kPBytes;
   static constexpr int kCtrlBytes = 4096;
   static constexpr int kSmemBytes = kOffCtrl + kCtrlBytes + 1024;   // + base alignment slack
   static constexpr uint32_t kPSwizzle = N == 64 ? 2u : (N == 32 ? 4u : 6u);   // 128/64/32 B
@@ -67,8 +69,8 @@ struct Cfg {
 };
 
 struct Ctrl {
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[16];
+  uint64_t empty[16];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
@@ -83,45 +85,6 @@ struct Ctrl {
   float lse_row[64];
   int kmax[64];           // keys < kmax[row] are visible in the current segment
   float red[4][64];       // cross-warp reduction scratch
-};
-
-// One (sequence, page range) piece of a part, as every role enumerates it.
-struct Seg {
-  int b, lo, hi, L, ntiles, piece;
-  bool ok;
-};
-
-struct SegIter {
-  int b, begin_b, begin_page, end_b, end_page, piece;
-
-  __device__ void init(const int32_t* md) {
-    begin_b = __ldg(md + 0);
-    begin_page = __ldg(md + 1);
-    end_b = __ldg(md + 2);
-    end_page = __ldg(md + 3);
-    piece = __ldg(md + 4);
-    b = begin_b;
-  }
-
-  __device__ bool next(const DecodeArgs& a, Seg& s) {
-    while (b < a.batch && (b < end_b || (b == end_b && end_page > 0))) {
-      const int cur = b++;
-      const int L = __ldg(a.seqlens + cur);
-      const int nb = L > 0 ? (L + 63) / 64 : 0;
-      const int lo = cur == begin_b ? begin_page : 0;
-      const int hi = cur == end_b ? end_page : nb;
-      if (hi <= lo) continue;
-      s.b = cur;
-      s.lo = lo;
-      s.L = L;
-      s.piece = piece++;
-      s.ok = L <= a.max_pages * 64 && hi <= nb;
-      s.hi = s.ok ? hi : lo;
-      s.ntiles = s.ok ? (hi - lo + 1) / 2 : 0;
-      return true;
-    }
-    return false;
-  }
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -205,22 +168,32 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
       return true;
     };
 
+    // pages two tiles ahead are pulled into L2 (one CTA of the row blocks and heads does it)
+    const bool prefetcher = rb == 0 && g == 0;
+    const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
+    auto prefetch_tile = [&](int t) {
+      if (!prefetcher || lane != 0) return;
+      for (int q = 0; q < 2; ++q) {
+        const int pg = s.lo + 2 * t + q;
+        if (pg >= s.hi) break;
+        const int id = __ldg(bt_row + pg);
+        if (id >= 0 && id < a.num_pages) l2_prefetch(a.k_cache + static_cast<size_t>(id) * page_bytes, page_bytes);
+      }
+    };
+
     auto issue_qk = [&](int t) -> bool {
       const int pid0 = page_id(s.lo + 2 * t), pid1 = page_id(s.lo + 2 * t + 1);
+      prefetch_tile(t + 2);
 #pragma unroll 1
-      for (int u = 0; u < 5; ++u) {
+      for (int c = 0; c < 9; ++c) {
         uint32_t slot;
         if (!acquire_slot(slot)) return false;
         if (lane == 0) {
+          // [page][64 tokens][64 cols]: the 128 keys of the tile contiguous, one column chunk
           uint8_t* dst = slots + slot * kSlotBytes;
-          const int nchunk = u < 4 ? 2 : 1;
-          mbar_arrive_expect_tx(&ct.full[slot], nchunk * 2 * kBoxBytes);
-          for (int j = 0; j < nchunk; ++j) {
-            // [chunk j][page][64 tokens][64 cols]: keys contiguous across the two pages
-            tma_load_3d(dst + j * 2 * kBoxBytes, tm_k, &ct.full[slot], 64 * (2 * u + j), g, 64 * pid0);
-            tma_load_3d(dst + j * 2 * kBoxBytes + kBoxBytes, tm_k, &ct.full[slot], 64 * (2 * u + j), g,
-                        64 * pid1);
-          }
+          mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
+          tma_load_3d(dst, tm_k, &ct.full[slot], 64 * c, g, 64 * pid0);
+          tma_load_3d(dst + kBoxBytes, tm_k, &ct.full[slot], 64 * c, g, 64 * pid1);
         }
         ++load_idx;
       }
@@ -230,24 +203,25 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
     auto issue_pv = [&](int t) -> bool {
       const int pid0 = page_id(s.lo + 2 * t), pid1 = page_id(s.lo + 2 * t + 1);
 #pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         uint32_t slot;
         if (!acquire_slot(slot)) return false;
         if (lane == 0) {
+          // [chunk j][64 tokens][64 cols] of one page: 128 dv columns of 64 keys
           uint8_t* dst = slots + slot * kSlotBytes;
-          mbar_arrive_expect_tx(&ct.full[slot], 4 * kBoxBytes);
-          for (int j = 0; j < 2; ++j) {
-            // [page][chunk j][64 tokens][64 cols]: 128 dv columns contiguous per page
-            tma_load_3d(dst + j * kBoxBytes, tm_k, &ct.full[slot], 64 * (2 * u + j), g, 64 * pid0);
-            tma_load_3d(dst + 2 * kBoxBytes + j * kBoxBytes, tm_k, &ct.full[slot], 64 * (2 * u + j), g,
-                        64 * pid1);
-          }
+          const int pid = (u & 1) ? pid1 : pid0;
+          const int col = 128 * (u >> 1);
+          mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
+          tma_load_3d(dst, tm_k, &ct.full[slot], col, g, 64 * pid);
+          tma_load_3d(dst + kBoxBytes, tm_k, &ct.full[slot], col + 64, g, 64 * pid);
         }
         ++load_idx;
       }
       return true;
     };
 
+    prefetch_tile(0);
+    prefetch_tile(1);
     if (!issue_qk(0)) { alive = false; break; }
 #pragma unroll 1
     for (int t = 1; t < s.ntiles && alive; ++t) {
@@ -304,19 +278,17 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
       tc_fence_after();
       const uint32_t d_tmem = tmem + 4 * N + sb * N;
 #pragma unroll 1
-      for (int u = 0; u < 5; ++u) {
+      for (int c = 0; c < 9; ++c) {
         const uint32_t slot = load_idx % C::kSlots;
         if (!wait_phase(&ct.full[slot], (load_idx / C::kSlots) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t base = slots_addr + slot * kSlotBytes;
-        const int nchunk = u < 4 ? 2 : 1;
-        for (int j = 0; j < nchunk; ++j) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(base + j * 2 * kBoxBytes + kk * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(q_addr + (2 * u + j) * N * 128 + kk * 32, 16, 1024, 2);
-            umma_bf16(d_tmem, ad, bd, idesc_qk, (u | j | kk) != 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 4; ++kk) {
+          // A = K: 128 keys x 16 columns, K-major; B = Q chunk c: N rows x 16 columns, K-major
+          const uint64_t ad = smem_desc(base + kk * 32, 16, 1024, 2);
+          const uint64_t bd = smem_desc(q_addr + c * N * 128 + kk * 32, 16, 1024, 2);
+          umma_bf16(d_tmem, ad, bd, idesc_qk, (c | kk) != 0 ? 1u : 0u);
         }
         umma_commit(&ct.empty[slot]);
         ++load_idx;
@@ -331,20 +303,21 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
       if (t == 0 && seg_i > 0 && !wait_phase(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
       if (!wait_phase(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
       tc_fence_after();
-      const uint32_t pbase = p_addr + pb * C::kPBytes;
+      const uint32_t pbase = p_addr + (tgl % C::kPBuf) * C::kPBytes;
 #pragma unroll 1
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint32_t slot = load_idx % C::kSlots;
         if (!wait_phase(&ct.full[slot], (load_idx / C::kSlots) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t base = slots_addr + slot * kSlotBytes;
+        const int q = u & 1;   // page of the tile: keys 64q .. 64q+63
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 4; ++kk) {
           // A = V^T: 128 dv (two 64-column boxes 8 KB apart) x 16 keys, MN-major
-          const uint64_t ad = smem_desc(base + (kk >> 2) * 2 * kBoxBytes + (kk & 3) * 2048, kBoxBytes, 1024, 2);
+          const uint64_t ad = smem_desc(base + kk * 2048, kBoxBytes, 1024, 2);
           // B = P^T: 16 keys x N rows, MN-major (rows contiguous)
-          const uint64_t bd = smem_desc(pbase + kk * 16 * 2 * N, C::kPBytes, 16 * N, C::kPSwizzle);
-          umma_bf16(tmem + u * N, ad, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = smem_desc(pbase + (4 * q + kk) * 16 * 2 * N, C::kPBytes, 16 * N, C::kPSwizzle);
+          umma_bf16(tmem + (u >> 1) * N, ad, bd, idesc_pv, (t > 0 || q > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&ct.empty[slot]);
         ++load_idx;
@@ -421,8 +394,9 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
     for (int t = 0; t < s.ntiles; ++t, ++tg) {
       const int sb = tg & 1;
       bool ok = wait_phase(&ct.s_full[sb], (tg >> 1) & 1, ctl);
-      // P buffer sb is free once the value product of tile tg-2 has finished
-      if (ok && tg >= 2) ok = wait_phase(&ct.p_free[sb], ((tg >> 1) - 1) & 1, ctl);
+      // the P buffer of this tile is free once the value product that last read it has finished
+      if (ok && tg >= C::kPBuf)
+        ok = wait_phase(&ct.p_free[(tg - C::kPBuf) & 1], ((tg - C::kPBuf) >> 1) & 1, ctl);
       float x[N];
       bool need = false;
       if (ok) {
@@ -491,7 +465,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
       }
 
       // P^T row of this key: N bf16 values, swizzled 16-byte chunks
-      uint8_t* pbuf = ps + sb * C::kPBytes;
+      uint8_t* pbuf = ps + (tg % C::kPBuf) * C::kPBytes;
 #pragma unroll
       for (int c8 = 0; c8 < N / 8; ++c8) {
         uint32_t w[4];
@@ -539,7 +513,6 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
     const bool final_out = npieces == 1;
     const bool can_write = final_out || s.piece < a.max_pieces;
     if (!can_write && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
-    float* stage_f = reinterpret_cast<float*>(ps);
     __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(ps);
 
 #pragma unroll 1
@@ -558,32 +531,30 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
 #pragma unroll
         for (int c = 0; c < N; ++c) v[c] = 0.f;
       }
-      // stage [row][128 dv] so each output row slice leaves as 16-byte vectors
       if (final_out) {
+        // stage [row][128 dv] bf16 (one P buffer) so each output row slice leaves as 16-byte vectors
 #pragma unroll
         for (int c = 0; c < N; ++c) stage_h[c * 128 + tid] = __float2bfloat16_rn(v[c] * ct.inv_l[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < N; ++c) stage_f[c * 128 + tid] = v[c] * ct.inv_l[c];
-      }
-      named_sync(kSoftmaxBar, 128);
-      if (can_write) {
-        const int vec_per_row = final_out ? 16 : 32;       // 16-byte vectors in 128 values
-        for (int i = tid; i < rows_here * vec_per_row; i += 128) {
-          const int c = i / vec_per_row, vv = i % vec_per_row;
-          const int r = rb * N + c;
-          const int srow = r / hg, h = g * hg + r % hg;
-          const uint4 val = reinterpret_cast<const uint4*>(ps)[c * vec_per_row + vv];
-          if (final_out) {
+        named_sync(kSoftmaxBar, 128);
+        if (can_write) {
+          for (int i = tid; i < rows_here * 16; i += 128) {
+            const int c = i >> 4, vv = i & 15;
+            const int r = rb * N + c;
+            const int srow = r / hg, h = g * hg + r % hg;
+            const uint4 val = reinterpret_cast<const uint4*>(ps)[c * 16 + vv];
             __nv_bfloat16* dst = a.out + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + h) * 512 + d * 128;
-            reinterpret_cast<uint4*>(dst)[vv] = val;
-          } else {
-            float* dst = a.o_part + ((static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + r) * 512 + d * 128;
             reinterpret_cast<uint4*>(dst)[vv] = val;
           }
         }
+        named_sync(kSoftmaxBar, 128);
+      } else if (can_write) {
+        // fp32 partials: a warp writes 32 consecutive floats (128 bytes) per row
+        float* dst = a.o_part + ((static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + rb * N) * 512 + d * 128 + tid;
+#pragma unroll
+        for (int c = 0; c < N; ++c) {
+          if (c < rows_here) dst[static_cast<size_t>(c) * 512] = v[c] * ct.inv_l[c];
+        }
       }
-      named_sync(kSoftmaxBar, 128);
     }
     if (tid < rows_here && can_write) {
       const int r = rb * N + tid;

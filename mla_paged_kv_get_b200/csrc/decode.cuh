@@ -10,6 +10,7 @@
 namespace mla {
 
 struct DecodeArgs {
+  const uint8_t* k_cache;       // [num_pages, 64, h_kv, 576] bf16 (bytes, for L2 prefetch)
   const int32_t* block_table;   // [batch, max_pages]
   const int32_t* seqlens;       // [batch]
   const int32_t* tile_md;       // [num_parts, 8]
@@ -29,6 +30,10 @@ struct DecodeArgs {
 int decode_smem_bytes(int rows_per_block);
 cudaError_t launch_decode(int rows_per_block, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                           const DecodeArgs& a, int row_blocks, cudaStream_t stream);
+
+int decode_pair_smem_bytes();
+cudaError_t launch_decode_pair(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, int row_blocks,
+                               cudaStream_t stream);
 
 cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
                            __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,

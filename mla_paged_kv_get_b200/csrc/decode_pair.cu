@@ -1,0 +1,605 @@
+// decode_pair.cu — split-KV MLA decode for 65..128 query rows per KV head, run
+// by CTA pairs (cluster of 2, tcgen05 cta_group::2) on B200.
+//
+// What it computes is the same as decode.cu (cnblogs "DeepSeek 开源记-第1天-
+// FlashMLA", §2 关键特性, §4.1 计算流程, §6.2 基本使用).  How:
+//   * A pair of CTAs (one per SM) drives one 2-SM MMA.  Each CTA keeps 64 query
+//     rows (72 KB) in shared memory: S = Q.K^T is one M = 128 x N = 128 x 576
+//     product per 128-key tile, the 128 keys being two 64-token pages of which
+//     each CTA loads one.  So every cache byte of the score product crosses
+//     L2 -> SM exactly once, and each SM reads only half of the B operand.
+//   * O = P.V in two M = 128 x N = 256 products (dv halves); each CTA supplies
+//     128 dv columns of both pages (a second, L2-hit read of half the latent
+//     columns) and receives the full P of its own 64 rows.
+//   * TMEM per CTA: O (2 x 128 columns: 64 rows x 512 dv in the pair layout
+//     that puts the second half of N in lanes 64..127) and two S buffers
+//     (64 columns each).  Thread t of warps 0-3 owns TMEM lane t: row
+//     t % 64 and key half (or dv quarter) t / 64, so the softmax of a row is
+//     split between two threads and needs no shuffles.
+//   * Separate load rings for the score product (one 8 KB box per slot) and
+//     for the value product (16 KB per slot), each with its own producer warp,
+//     so value loads for tile t overlap the score product of tile t+1.
+//   * The leader CTA (rank 0) issues every MMA; the peer's TMA loads complete
+//     on the leader's barriers (cta_group::2 loads, no multicast), MMA
+//     completions are committed to both CTAs, and the peer's softmax warps
+//     arrive on the leader's barriers through cluster shared memory.
+//   * Online softmax in log2 units with the lazy rescale of decode.cu (TAU = 8),
+//     every wait bounded; an expired wait records MLA_ERR_TIMEOUT and the pair
+//     unwinds.
+#include <float.h>
+
+#include "ptx.cuh"
+#include "decode.cuh"
+#include "segments.cuh"
+
+namespace mla {
+
+namespace {
+
+constexpr int kRows = 64;              // query rows per CTA
+constexpr int kBox = 8192;             // one TMA box: 64 tokens x 64 bf16 columns
+constexpr int kKSlots = 6;             // score ring: one box per slot
+constexpr int kVSlots = 4;             // value ring: two boxes (128 dv of one page) per slot
+constexpr int kThreads = 224;          // warps 0-3 softmax, 4 score loads, 5 value loads, 6 MMA
+constexpr int kQBytes = 9 * kBox;      // 64 rows x 576
+constexpr int kPBytes = 2 * kBox;      // P: [key half][64 rows][64 keys] bf16
+constexpr int kOffP = kQBytes;
+constexpr int kOffK = kOffP + 2 * kPBytes;
+constexpr int kOffV = kOffK + kKSlots * kBox;
+constexpr int kOffCtrl = kOffV + kVSlots * 2 * kBox;
+constexpr int kSmemBytes = kOffCtrl + 4096 + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColO = 0;               // O half h at column 128 h
+constexpr int kColS = 256;             // S buffer b at column 256 + 64 b
+constexpr float kTau = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kSoftmaxBar = 1;
+
+struct Ctrl {
+  uint64_t k_full[kKSlots], k_empty[kKSlots];
+  uint64_t v_full[kVSlots], v_empty[kVSlots];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], p_free[2];
+  uint64_t o_free, never, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int softmax_abort;
+  int pad;
+  float red[2][kRows];    // [key half][row] scratch shared by the two threads of a row
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void settle_ns(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) {
+  }
+}
+
+// Page ids of the current sequence, 32 at a time, one per lane of the warp.
+struct PageWindow {
+  const int32_t* row;
+  int hi, base, val, num_pages;
+  int32_t* status;
+
+  __device__ void reset(const int32_t* r, int h, int np, int32_t* st) {
+    row = r;
+    hi = h;
+    base = -1;
+    val = 0;
+    num_pages = np;
+    status = st;
+  }
+  // All 32 lanes call this with the same `pg`.
+  __device__ int get(int pg) {
+    const int lane = threadIdx.x & 31;
+    const int b = pg & ~31;
+    if (b != base) {
+      base = b;
+      const int idx = b + lane;
+      val = idx < hi ? __ldg(row + idx) : num_pages;
+    }
+    int v = __shfl_sync(0xffffffffu, val, pg & 31);
+    if (pg >= hi) return num_pages;               // absent second page: zero-filled box
+    if (v < 0 || v >= num_pages) {                // corrupt id: never read out of bounds
+      if (lane == 0) record_status(status, MLA_ERR_BAD_INPUT);
+      v = num_pages;
+    }
+    return v;
+  }
+};
+
+// ------------------------------------------------------------------ loads
+// Warp 4: Q at each segment start, then the nine 64-column boxes of this CTA's
+// page of every tile, for the score product.
+__device__ void score_loads(const CUtensorMap* tm_k, const CUtensorMap* tm_q, const DecodeArgs& a, Ctrl& ct,
+                            uint8_t* qs, uint8_t* ks, const Ctl& ctl, uint32_t rank, int rb, int g,
+                            const int32_t* md, uint32_t leader_q_full, uint32_t leader_k_full0) {
+  const int lane = threadIdx.x & 31;
+  const int hg = a.hg;
+  const int r0 = rb * kRows;
+  const int q_h0 = hg >= kRows ? r0 % hg : 0;
+  const int q_s0 = r0 / hg;
+  const bool leader = rank == 0;
+  const bool prefetcher = leader && g == 0;
+  const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
+  uint32_t kidx = 0;
+  int qloads = 0;
+  bool alive = true;
+  auto wait_uniform = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 1;
+    if (lane == 0) ok = wait_phase(bar, parity, ctl) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+  SegIter it;
+  it.init(md);
+  Seg s;
+  PageWindow win;
+  while (alive && it.next(a, s)) {
+    if (s.ntiles == 0) continue;
+    if (qloads > 0 && !wait_uniform(&ct.q_empty, (qloads - 1) & 1)) { alive = false; break; }
+    if (lane == 0) {
+      if (leader) mbar_arrive_expect_tx(&ct.q_full, 2 * kQBytes);
+      for (int c = 0; c < 9; ++c)
+        tma_load_4d_pair(qs + c * kBox, tm_q, leader_q_full, 64 * c, q_h0, g, s.b * a.s_q + q_s0);
+    }
+    ++qloads;
+    const int32_t* bt_row = a.block_table + static_cast<size_t>(s.b) * a.max_pages;
+    win.reset(bt_row, s.hi, a.num_pages, a.status);
+    auto prefetch_tile = [&](int t) {
+      if (!prefetcher || lane != 0) return;
+      for (int q = 0; q < 2; ++q) {
+        const int pg = s.lo + 2 * t + q;
+        if (pg >= s.hi) break;
+        const int id = __ldg(bt_row + pg);
+        if (id >= 0 && id < a.num_pages) l2_prefetch(a.k_cache + static_cast<size_t>(id) * page_bytes, page_bytes);
+      }
+    };
+    prefetch_tile(0);
+    prefetch_tile(1);
+#pragma unroll 1
+    for (int t = 0; t < s.ntiles && alive; ++t) {
+      const int pid = win.get(s.lo + 2 * t + static_cast<int>(rank));
+      prefetch_tile(t + 2);
+#pragma unroll 1
+      for (int c = 0; c < 9; ++c) {
+        const uint32_t slot = kidx % kKSlots;
+        if (kidx >= static_cast<uint32_t>(kKSlots) && !wait_uniform(&ct.k_empty[slot], ((kidx / kKSlots) - 1) & 1)) {
+          alive = false;
+          break;
+        }
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&ct.k_full[slot], 2 * kBox);
+          tma_load_3d_pair(ks + slot * kBox, tm_k, leader_k_full0 + slot * 8, 64 * c, g, 64 * pid);
+        }
+        ++kidx;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// Warp 5: for the value product of every tile, this CTA's 128 dv columns of each
+// dv half, for both pages: [page q][dv half h] -> one 16 KB slot [box j][64 tokens][64 cols].
+__device__ void value_loads(const CUtensorMap* tm_k, const DecodeArgs& a, Ctrl& ct, uint8_t* vs, const Ctl& ctl,
+                            uint32_t rank, int g, const int32_t* md, uint32_t leader_v_full0) {
+  const int lane = threadIdx.x & 31;
+  const bool leader = rank == 0;
+  uint32_t vidx = 0;
+  bool alive = true;
+  auto wait_uniform = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 1;
+    if (lane == 0) ok = wait_phase(bar, parity, ctl) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+  SegIter it;
+  it.init(md);
+  Seg s;
+  PageWindow win;
+  while (alive && it.next(a, s)) {
+    if (s.ntiles == 0) continue;
+    win.reset(a.block_table + static_cast<size_t>(s.b) * a.max_pages, s.hi, a.num_pages, a.status);
+#pragma unroll 1
+    for (int t = 0; t < s.ntiles && alive; ++t) {
+      const int pid0 = win.get(s.lo + 2 * t), pid1 = win.get(s.lo + 2 * t + 1);
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {     // u = 2 h + q
+        const int h = u >> 1, q = u & 1;
+        const uint32_t slot = vidx % kVSlots;
+        if (vidx >= static_cast<uint32_t>(kVSlots) && !wait_uniform(&ct.v_empty[slot], ((vidx / kVSlots) - 1) & 1)) {
+          alive = false;
+          break;
+        }
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&ct.v_full[slot], 4 * kBox);
+          const int col = 256 * h + 128 * static_cast<int>(rank);
+          const int pid = q ? pid1 : pid0;
+          uint8_t* dst = vs + slot * 2 * kBox;
+          tma_load_3d_pair(dst, tm_k, leader_v_full0 + slot * 8, col, g, 64 * pid);
+          tma_load_3d_pair(dst + kBox, tm_k, leader_v_full0 + slot * 8, col + 64, g, 64 * pid);
+        }
+        ++vidx;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------------ MMA (leader CTA, one thread)
+__device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* ps, uint8_t* ks, uint8_t* vs,
+                          uint32_t tmem, const Ctl& ctl, const int32_t* md) {
+  const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);   // A = Q (K-major), B = K (K-major)
+  const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);    // A = P (K-major), B = V (MN-major)
+  const uint32_t q_addr = smem_addr(qs), p_addr = smem_addr(ps), k_addr = smem_addr(ks), v_addr = smem_addr(vs);
+  uint32_t kidx = 0, vidx = 0;
+  int tg = 0, qloads = 0, seg_i = 0;
+  SegIter it;
+  it.init(md);
+  Seg s;
+  while (it.next(a, s)) {
+    const int tg0 = tg;
+    if (s.ntiles == 0) {
+      if (seg_i > 0 && !wait_phase_cluster(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
+      ++seg_i;
+      continue;
+    }
+    if (!wait_phase(&ct.q_full, qloads & 1, ctl)) return false;
+    ++qloads;
+    tc_fence_after();
+
+    auto do_qk = [&](int t) -> bool {
+      const int tgl = tg0 + t, sb = tgl & 1;
+      if (tgl >= 2 && !wait_phase_cluster(&ct.s_free[sb], ((tgl >> 1) - 1) & 1, ctl)) return false;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + kColS + 64 * sb;
+#pragma unroll 1
+      for (int c = 0; c < 9; ++c) {
+        const uint32_t slot = kidx % kKSlots;
+        if (!wait_phase(&ct.k_full[slot], (kidx / kKSlots) & 1, ctl)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc(q_addr + c * kBox + kk * 32, 16, 1024, 2);
+          const uint64_t bd = smem_desc(k_addr + slot * kBox + kk * 32, 16, 1024, 2);
+          umma_bf16_pair(d_tmem, ad, bd, idesc_qk, (c | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit_pair(&ct.k_empty[slot]);
+        ++kidx;
+      }
+      umma_commit_pair(&ct.s_full[sb]);
+      if (t == s.ntiles - 1) umma_commit_pair(&ct.q_empty);
+      return true;
+    };
+
+    auto do_pv = [&](int t) -> bool {
+      const int tgl = tg0 + t, pb = tgl & 1;
+      if (t == 0 && seg_i > 0 && !wait_phase_cluster(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
+      if (!wait_phase_cluster(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int u = 0; u < 4; ++u) {       // u = 2 h + q: dv half h, page q of the tile
+        const int h = u >> 1, q = u & 1;
+        const uint32_t slot = vidx % kVSlots;
+        if (!wait_phase(&ct.v_full[slot], (vidx / kVSlots) & 1, ctl)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // A = P: 128 rows (64 per CTA) x 16 keys of page q, K-major
+          const uint64_t ad = smem_desc(p_addr + pb * kPBytes + q * kBox + kk * 32, 16, 1024, 2);
+          // B = V: 16 keys x 256 dv (128 per CTA: two boxes 8 KB apart), MN-major
+          const uint64_t bd = smem_desc(v_addr + slot * 2 * kBox + kk * 2048, kBox, 1024, 2);
+          umma_bf16_pair(tmem + kColO + 128 * h, ad, bd, idesc_pv, (t > 0 || q > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit_pair(&ct.v_empty[slot]);
+        ++vidx;
+      }
+      umma_commit_pair(&ct.p_free[pb]);
+      return true;
+    };
+
+    if (!do_qk(0)) return false;
+#pragma unroll 1
+    for (int t = 1; t < s.ntiles; ++t) {
+      if (!do_qk(t) || !do_pv(t - 1)) return false;
+    }
+    if (!do_pv(s.ntiles - 1)) return false;
+    tg += s.ntiles;
+    ++seg_i;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ softmax + epilogue (warps 0-3)
+__device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_t tmem, const Ctl& ctl,
+                             uint32_t rank, int rb, int g, const int32_t* md, uint32_t leader_s_free0,
+                             uint32_t leader_p_full0, uint32_t leader_o_free) {
+  const int tid = threadIdx.x;                 // TMEM lane
+  const int warp = tid >> 5, lane = tid & 31;
+  const int r = tid & 63, kh = tid >> 6;       // row of this CTA, key half / dv quarter
+  const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+  const int rr = rb * kRows + r;               // row within the KV head group
+  const bool row_valid = rr < a.R;
+  const int hg = a.hg;
+  const int srow = row_valid ? rr / hg : 0;
+  const int head = g * hg + (row_valid ? rr % hg : 0);
+
+  auto uniform_ok = [&](bool ok) -> bool {
+    if (!ok) ct.softmax_abort = 1;
+    named_sync(kSoftmaxBar, 128);
+    return ct.softmax_abort == 0;
+  };
+  if (a.debug_flags & 1) {
+    if (!uniform_ok(wait_phase(&ct.never, 0, ctl))) return;
+  }
+
+  int tg = 0;
+  SegIter it;
+  it.init(md);
+  Seg s;
+  while (it.next(a, s)) {
+    int kmax = 0;
+    if (row_valid && s.ok) {
+      const int seg_end = min(s.hi * 64, s.L);
+      const int lim = a.causal ? s.L - (a.s_q - 1 - srow) : s.L;
+      kmax = min(seg_end, lim);
+    }
+    if (!s.ok && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
+    float m_run = -INFINITY, lsum = 0.f;
+
+#pragma unroll 1
+    for (int t = 0; t < s.ntiles; ++t, ++tg) {
+      const int sb = tg & 1;
+      bool ok = wait_phase(&ct.s_full[sb], (tg >> 1) & 1, ctl);
+      if (ok && tg >= 2) ok = wait_phase(&ct.p_free[sb], ((tg >> 1) - 1) & 1, ctl);   // P buffer sb free
+      float x[64];
+      bool need = false;
+      float mloc = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + kColS + 64 * sb + 16 * c16, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[16 * c16 + i] = __uint_as_float(v[i]);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_s_free0 + sb * 8);
+        const int key0 = (s.lo + 2 * t) * 64 + 64 * kh;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = key0 + j < kmax ? x[j] * a.scale_log2 : -INFINITY;
+          mloc = fmaxf(mloc, x[j]);
+        }
+        need = mloc > m_run + kTau;
+      }
+      if (!ok) ct.softmax_abort = 1;
+      need = named_sync_or(kSoftmaxBar, 128, need);
+      if (ct.softmax_abort) return;
+
+      if (need) {
+        ct.red[kh][r] = mloc;
+        named_sync(kSoftmaxBar, 128);
+        const float mt = fmaxf(ct.red[0][r], ct.red[1][r]);
+        const float mn = fmaxf(m_run, mt);
+        const float alpha = m_run == -INFINITY ? (mn == -INFINITY ? 1.f : 0.f) : ex2(m_run - mn);
+        m_run = mn;
+        lsum *= alpha;
+        if (t > 0) {
+          const bool okr = wait_phase(&ct.p_free[(tg - 1) & 1], ((tg - 1) >> 1) & 1, ctl);
+          if (!uniform_ok(okr)) return;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c16 = 0; c16 < 16; ++c16) {     // this lane's 256 O columns (both dv halves)
+            uint32_t v[16];
+            const uint32_t ta = tmem + lane_base + kColO + 16 * c16;
+            tmem_ld16(ta, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st16(ta, v);
+          }
+          tmem_wait_st();
+        }
+        named_sync(kSoftmaxBar, 128);              // red[] is reused by the next tile
+      }
+
+      // P row slice: 64 keys of this thread's half, 128 bytes, 128-byte swizzle
+      uint8_t* prow = ps + (tg & 1) * kPBytes + kh * kBox + r * 128;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 8 * c8 + 2 * i;
+          const float p0 = x[j] == -INFINITY ? 0.f : ex2(x[j] - m_run);
+          const float p1 = x[j + 1] == -INFINITY ? 0.f : ex2(x[j + 1] - m_run);
+          w[i] = pack_bf16(p0, p1);
+          lsum += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+        }
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_p_full0 + (tg & 1) * 8);
+    }
+
+    // ---------------- epilogue of the segment
+    if (s.ntiles > 0) {
+      const int tl = tg - 1;
+      const bool okw = wait_phase(&ct.p_free[tl & 1], (tl >> 1) & 1, ctl);
+      if (!uniform_ok(okw)) return;
+      tc_fence_after();
+    }
+    ct.red[kh][r] = lsum;
+    named_sync(kSoftmaxBar, 128);
+    const float l = ct.red[0][r] + ct.red[1][r];
+    const bool any = l > 0.f;
+    const float inv = any ? 1.f / l : 0.f;
+    const float lse = any ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+    named_sync(kSoftmaxBar, 128);
+
+    const int npieces = __ldg(a.num_splits + s.b + 1) - __ldg(a.num_splits + s.b);
+    const bool final_out = npieces == 1;
+    const bool can_write = row_valid && (final_out || s.piece < a.max_pieces);
+    if (!final_out && s.piece >= a.max_pieces && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      float v[128];
+      if (s.ntiles > 0) {
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t u[16];
+          tmem_ld16(tmem + lane_base + kColO + 128 * h + 16 * c16, u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[16 * c16 + i] = __uint_as_float(u[i]) * inv;
+        }
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) v[i] = 0.f;
+      }
+      if (can_write) {
+        const int dv0 = 256 * h + 128 * kh;   // this thread's 128 contiguous dv values of its row
+        if (final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(
+              a.out + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + head) * 512 + dv0);
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            dst[k] = make_uint4(pack_bf16(v[8 * k], v[8 * k + 1]), pack_bf16(v[8 * k + 2], v[8 * k + 3]),
+                                pack_bf16(v[8 * k + 4], v[8 * k + 5]), pack_bf16(v[8 * k + 6], v[8 * k + 7]));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(
+              a.o_part + ((static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + rr) * 512 + dv0);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        }
+      }
+    }
+    if (kh == 0 && can_write) {
+      if (final_out)
+        a.lse[(static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + head] = lse;
+      else
+        a.lse_part[(static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + rr] = lse;
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(leader_o_free);
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                       const DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* qs = smem;
+  uint8_t* ps = smem + kOffP;
+  uint8_t* ks = smem + kOffK;
+  uint8_t* vs = smem + kOffV;
+  Ctrl& ct = *reinterpret_cast<Ctrl*>(smem + kOffCtrl);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const int rb = blockIdx.x;                    // row block of 64 rows; the pair is (2i, 2i+1)
+  const int g = blockIdx.y, part = blockIdx.z;
+  const int32_t* md = a.tile_md + static_cast<size_t>(part) * MLA_MD_WORDS;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kKSlots; ++i) {
+      mbar_init(&ct.k_full[i], 1);
+      mbar_init(&ct.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
+      mbar_init(&ct.v_full[i], 1);
+      mbar_init(&ct.v_empty[i], 1);
+    }
+    mbar_init(&ct.q_full, 1);
+    mbar_init(&ct.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ct.s_full[i], 1);
+      mbar_init(&ct.s_free[i], 8);    // one arrival per softmax warp of both CTAs
+      mbar_init(&ct.p_full[i], 8);
+      mbar_init(&ct.p_free[i], 1);
+    }
+    mbar_init(&ct.o_free, 8);
+    mbar_init(&ct.never, 1);
+    mbar_init(&ct.drain, 1);
+    ct.abort_flag = 0;
+    ct.softmax_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 6) {
+    tmem_alloc_pair(&ct.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 4 && (threadIdx.x & 31) == 0) {
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_q);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();           // barriers of both CTAs initialised before any remote arrive or load
+  tc_fence_after();
+  const uint32_t tmem = ct.tmem_base;
+  const Ctl ctl{&ct.abort_flag, a.status, a.timeout_ns};
+  // barriers of the leader CTA, in the cluster shared window
+  const uint32_t L_q_full = mapa_shared(smem_addr(&ct.q_full), 0);
+  const uint32_t L_k_full0 = mapa_shared(smem_addr(&ct.k_full[0]), 0);
+  const uint32_t L_v_full0 = mapa_shared(smem_addr(&ct.v_full[0]), 0);
+  const uint32_t L_s_free0 = mapa_shared(smem_addr(&ct.s_free[0]), 0);
+  const uint32_t L_p_full0 = mapa_shared(smem_addr(&ct.p_full[0]), 0);
+  const uint32_t L_o_free = mapa_shared(smem_addr(&ct.o_free), 0);
+
+  bool clean = true;
+  if (warp < 4) {
+    softmax_rows(a, ct, ps, tmem, ctl, rank, rb, g, md, L_s_free0, L_p_full0, L_o_free);
+  } else if (warp == 4) {
+    score_loads(&tm_k, &tm_q, a, ct, qs, ks, ctl, rank, rb, g, md, L_q_full, L_k_full0);
+  } else if (warp == 5) {
+    value_loads(&tm_k, a, ct, vs, ctl, rank, g, md, L_v_full0);
+  } else if (rank == 0 && (threadIdx.x & 31) == 0) {
+    clean = mma_issue(a, ct, qs, ps, ks, vs, tmem, ctl, md);
+    if (!clean) {
+      umma_commit_pair(&ct.drain);      // every MMA issued so far has finished before TMEM is freed
+      drain_phase(&ct.drain, 0, 1000000000ull);
+    }
+  }
+  __syncthreads();
+  if (ct.abort_flag) settle_ns(200000);   // let loads already issued land before the pair exits
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 6) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int decode_pair_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_decode_pair(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, int row_blocks,
+                               cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  const int pairs = (row_blocks + 1) / 2;
+  const dim3 grid(2 * pairs, a.h_kv, a.num_parts);
+  mla_decode_pair_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, a);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

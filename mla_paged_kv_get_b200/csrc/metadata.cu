@@ -4,19 +4,22 @@
 // takes the sequence lengths, s_q*h_q/h_kv and h_kv and returns the scheduler
 // table and num_splits).
 //
-// The rule (integer-only, so the table is bit-exact and deterministic):
-//   n_b = ceil(L_b / 64) pages, cost c_b = n_b + C (0 for an empty sequence),
-//   C = 4 pages of per-piece overhead, capacity W = ceil(sum c_b / G) + C.
-//   Parts 0..G-2 are filled in order from a (sequence, page) cursor: skip
-//   empty sequences; take the rest of a sequence while rest + C <= remaining;
-//   otherwise take remaining - C pages (if >= 1) and close the part.  The last
-//   part takes everything left.  Entry p = (begin_b, begin_page, end_b,
-//   end_page, first_piece, n_pieces, 0, 0), end exclusive; pieces are numbered
-//   in sweep order and num_splits is the prefix sum of pieces per sequence.
+// The rule (integer-only, so the table is bit-exact and deterministic) is a
+// partition of a cost line:
+//   sequence b with n_b = ceil(L_b / 64) pages occupies c_b = C + n_b units
+//   (0 if empty): C = 4 overhead units, then one unit per page.  P_b is the
+//   prefix sum of c_b, W = max(1, ceil(total / G)); part p owns units
+//   [p*W, (p+1)*W) (the last part everything after (G-1)*W), and page j of
+//   sequence b goes to the part that owns unit P_b + C + j.
+//   pos(U) = first (sequence, page) whose unit is >= U, or (B, 0).  Entry p is
+//   (pos(p*W), pos((p+1)*W) or (B,0) for the last part, first_piece,
+//   n_pieces, 0, 0); a piece is a (part, sequence) pair with >= 1 page,
+//   numbered part by part; num_splits is the prefix sum of pieces per
+//   sequence.
 //
-// One CTA: all threads compute page counts and the total cost, one thread
-// sweeps (G + batch steps out of shared memory), all threads scan the piece
-// counts into num_splits.
+// Every part and every sequence is independent given the prefix sums, so one
+// CTA does it with three block scans and one binary search per part: no
+// sequential sweep.
 #include "decode.cuh"
 
 namespace mla {
@@ -24,138 +27,166 @@ namespace mla {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kOverheadPages = 4;
+constexpr int kWarps = kThreads / 32;
+constexpr int kOverhead = 4;
+constexpr int kMaxBatch = 8192;
+constexpr int kMaxParts = 4096;
+
+// Exclusive prefix of `v` over the CTA (thread order); `*total` gets the sum.
+__device__ long long block_exclusive_scan(long long v, long long* warp_buf, long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const long long w = warp_buf[lane];
+    long long x = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    warp_buf[lane] = x - w;
+    if (lane == 31) warp_buf[32] = x;
+  }
+  __syncthreads();
+  const long long r = warp_buf[warp] + incl - v;
+  *total = warp_buf[32];
+  __syncthreads();
+  return r;
+}
+
+struct Pos {
+  int b, page;
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_parts,
                     int32_t* __restrict__ tile_md, int32_t* __restrict__ num_splits) {
-  extern __shared__ int smem_i[];
-  int* n_s = smem_i;              // pages per sequence
-  int* pieces = smem_i + batch;   // pieces per sequence
-  __shared__ long long warp_tot[32];
-  __shared__ int warp_scan[32];
-  __shared__ long long total_s;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ long long smem_ll[];
+  long long* p_incl = smem_ll;                                        // [batch]  P_{b+1}
+  int* n_s = reinterpret_cast<int*>(p_incl + batch);                  // [batch]  pages
+  int* ne_s = n_s + batch;                                            // [batch+1] non-empty before b
+  int* np_s = ne_s + batch + 1;                                       // [num_parts] pieces per part
+  __shared__ long long warp_buf[33];
+  const int tid = threadIdx.x;
 
-  long long local = 0;
-  for (int b = tid; b < batch; b += kThreads) {
+  // ---- prefix sums of cost and of non-empty sequences (contiguous chunk per thread)
+  const int per = (batch + kThreads - 1) / kThreads;
+  const int b0 = min(tid * per, batch), b1 = min(b0 + per, batch);
+  long long my_cost = 0;
+  int my_ne = 0;
+  for (int b = b0; b < b1; ++b) {
     const int L = __ldg(seqlens + b);
     const int nb = L > 0 ? (L + 63) / 64 : 0;
     n_s[b] = nb;
-    pieces[b] = 0;
-    if (nb > 0) local += nb + kOverheadPages;
+    my_cost += nb > 0 ? nb + kOverhead : 0;
+    my_ne += nb > 0;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  if (lane == 0) warp_tot[warp] = local;
-  __syncthreads();
-  if (tid == 0) {
-    long long t = 0;
-    for (int w = 0; w < kThreads / 32; ++w) t += warp_tot[w];
-    total_s = t;
+  long long total_cost, total_ne;
+  long long run = block_exclusive_scan(my_cost, warp_buf, &total_cost);
+  long long run_ne = block_exclusive_scan(my_ne, warp_buf, &total_ne);
+  for (int b = b0; b < b1; ++b) {
+    const int nb = n_s[b];
+    ne_s[b] = static_cast<int>(run_ne);
+    run += nb > 0 ? nb + kOverhead : 0;
+    run_ne += nb > 0;
+    p_incl[b] = run;
   }
-  __syncthreads();
-
-  if (tid == 0) {
-    const long long G = num_parts;
-    const long long W = (total_s + G - 1) / G + kOverheadPages;
-    int b = 0, page = 0, piece = 0;
-    for (int p = 0; p < num_parts; ++p) {
-      const int begin_b = b, begin_page = page, first_piece = piece;
-      if (p == num_parts - 1) {
-        while (b < batch) {
-          if (n_s[b] > page) {
-            ++pieces[b];
-            ++piece;
-          }
-          ++b;
-          page = 0;
-        }
-      } else {
-        long long remaining = W;
-        while (b < batch) {
-          const int nb = n_s[b];
-          if (nb == 0) {
-            ++b;
-            page = 0;
-            continue;
-          }
-          const int rest = nb - page;
-          if (rest + kOverheadPages <= remaining) {
-            remaining -= rest + kOverheadPages;
-            ++pieces[b];
-            ++piece;
-            ++b;
-            page = 0;
-          } else {
-            const long long take = remaining - kOverheadPages;
-            if (take >= 1) {
-              page += static_cast<int>(take);
-              ++pieces[b];
-              ++piece;
-            }
-            break;
-          }
-        }
-      }
-      int32_t* row = tile_md + static_cast<size_t>(p) * 8;
-      row[0] = begin_b;
-      row[1] = begin_page;
-      row[2] = b;
-      row[3] = page;
-      row[4] = first_piece;
-      row[5] = piece - first_piece;
-      row[6] = 0;
-      row[7] = 0;
-    }
-  }
+  if (tid == 0) ne_s[batch] = static_cast<int>(total_ne);
   __syncthreads();
 
-  // exclusive scan of pieces -> num_splits[0..batch]
-  const int per = (batch + kThreads - 1) / kThreads;
-  const int start = min(tid * per, batch), end = min(start + per, batch);
-  int mine = 0;
-  for (int i = start; i < end; ++i) mine += pieces[i];
-  int incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_scan[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int v = warp_scan[lane];
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+  const long long G = num_parts;
+  const long long W = total_cost > 0 ? (total_cost + G - 1) / G : 1;
+
+  auto pos = [&](long long U) -> Pos {
+    if (U >= total_cost) return Pos{batch, 0};
+    int lo = 0, hi = batch - 1;            // first b with p_incl[b] > U
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (p_incl[mid] > U) hi = mid; else lo = mid + 1;
     }
-    warp_scan[lane] = x - v;   // exclusive prefix over warps
+    const long long start = lo > 0 ? p_incl[lo - 1] : 0;
+    const long long pg = U - start - kOverhead;
+    return Pos{lo, pg > 0 ? static_cast<int>(pg) : 0};
+  };
+  auto part_of = [&](long long unit) -> int {
+    const long long p = unit / W;
+    return static_cast<int>(p < G - 1 ? p : G - 1);
+  };
+
+  // ---- parts: boundaries and piece counts
+  for (int p = tid; p < num_parts; p += kThreads) {
+    const Pos be = pos(static_cast<long long>(p) * W);
+    const Pos en = p < num_parts - 1 ? pos(static_cast<long long>(p + 1) * W) : Pos{batch, 0};
+    const bool empty = be.b == en.b && be.page == en.page;
+    np_s[p] = empty ? 0 : ne_s[en.b] - ne_s[be.b] + (en.page > 0 ? 1 : 0);
+    int32_t* row = tile_md + static_cast<size_t>(p) * 8;
+    row[0] = be.b;
+    row[1] = be.page;
+    row[2] = en.b;
+    row[3] = en.page;
+    row[6] = 0;
+    row[7] = 0;
   }
-  __syncthreads();
-  int run = warp_scan[warp] + incl - mine;
-  for (int i = start; i < end; ++i) {
-    num_splits[i] = run;
-    run += pieces[i];
+
+  // ---- pieces per sequence -> num_splits
+  long long my_pieces = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int nb = n_s[b];
+    if (nb > 0) {
+      const long long first_unit = (b > 0 ? p_incl[b - 1] : 0) + kOverhead;
+      my_pieces += part_of(first_unit + nb - 1) - part_of(first_unit) + 1;
+    }
   }
-  if (tid == kThreads - 1) num_splits[batch] = warp_scan[warp] + incl;
+  long long total_pieces;
+  long long run_p = block_exclusive_scan(my_pieces, warp_buf, &total_pieces);
+  for (int b = b0; b < b1; ++b) {
+    num_splits[b] = static_cast<int32_t>(run_p);
+    const int nb = n_s[b];
+    if (nb > 0) {
+      const long long first_unit = (b > 0 ? p_incl[b - 1] : 0) + kOverhead;
+      run_p += part_of(first_unit + nb - 1) - part_of(first_unit) + 1;
+    }
+  }
+  if (tid == 0) num_splits[batch] = static_cast<int32_t>(total_pieces);
+
+  // ---- first piece of each part: prefix over parts (contiguous chunk per thread)
+  const int pper = (num_parts + kThreads - 1) / kThreads;
+  const int p0 = min(tid * pper, num_parts), p1 = min(p0 + pper, num_parts);
+  long long my_np = 0;
+  for (int p = p0; p < p1; ++p) my_np += np_s[p];
+  long long total_np;
+  long long run_np = block_exclusive_scan(my_np, warp_buf, &total_np);
+  for (int p = p0; p < p1; ++p) {
+    int32_t* row = tile_md + static_cast<size_t>(p) * 8;
+    row[4] = static_cast<int32_t>(run_np);
+    row[5] = np_s[p];
+    run_np += np_s[p];
+  }
 }
 
 }  // namespace
 
-int metadata_max_batch() { return 16384; }
+int metadata_max_batch() { return kMaxBatch; }
+int metadata_max_parts() { return kMaxParts; }
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,
                             int32_t* num_splits, cudaStream_t stream) {
-  const int smem = 2 * batch * static_cast<int>(sizeof(int));
+  const size_t smem = static_cast<size_t>(batch) * sizeof(long long) + (2 * batch + 1) * sizeof(int) +
+                      static_cast<size_t>(num_parts) * sizeof(int);
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         2 * metadata_max_batch() * static_cast<int>(sizeof(int)));
+    const int max_smem = kMaxBatch * static_cast<int>(sizeof(long long)) +
+                         (2 * kMaxBatch + 1) * static_cast<int>(sizeof(int)) + kMaxParts * static_cast<int>(sizeof(int));
+    cudaError_t e = cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }

@@ -12,19 +12,22 @@ this project's reading, stated in full in DESIGN.md ("Scheduler rule"):
 
 * rows per KV head ``R = s_q*h_q/h_kv`` are cut into row blocks of
   ``N = 16`` (R <= 16), ``32`` (R <= 32) or ``64`` rows; ``T = ceil(R/N)``;
-* ``G = max(1, num_sms // (h_kv*T))`` parts; each part is one CTA per
-  (row block, KV head);
-* sequence ``b`` has ``n_b = ceil(L_b/64)`` pages and costs
-  ``c_b = n_b + C`` (0 if empty), ``C = 4`` pages of per-piece overhead;
-* capacity ``W = ceil(sum_b c_b / G) + C``;
-* parts ``0..G-2`` are filled in order: whole sequences while
-  ``rest + C <= remaining``; otherwise ``remaining - C`` pages of the
-  current sequence (if that is at least 1) and the part closes;
-* the last part takes everything left;
-* ``tile_md[p] = (begin_b, begin_page, end_b, end_page, first_piece,
-  n_pieces, 0, 0)`` with the end exclusive in (sequence, page) order;
-* pieces are numbered in sweep order; ``num_splits`` is the prefix sum of the
-  number of pieces per sequence (length ``B + 1``).
+* ``G = max(1, num_sms // (h_kv*T))`` parts;
+* the cost line: sequence ``b`` with ``n_b = ceil(L_b/64)`` pages occupies
+  ``c_b = C + n_b`` units (0 if empty), ``C = 4`` units of per-sequence
+  overhead first, then one unit per page; ``P_b`` is the prefix sum of the
+  ``c_b`` and ``total = P_B``;
+* ``W = max(1, ceil(total / G))``; part ``p`` owns units ``[p*W, (p+1)*W)``,
+  the last part everything from ``(G-1)*W`` on;
+* page ``j`` of sequence ``b`` goes to the part owning unit ``P_b + C + j``;
+* ``pos(U)``: the first (sequence, page) whose unit is ``>= U`` (``(B, 0)``
+  past the end); ``tile_md[p] = (begin_b, begin_page, end_b, end_page,
+  first_piece, n_pieces, 0, 0)`` with ``begin = pos(p*W)`` and
+  ``end = pos((p+1)*W)`` (``(B, 0)`` for the last part), end exclusive;
+* a piece is a (part, sequence) pair with at least one page; pieces are
+  numbered part by part, sequences in order within a part; ``first_piece``
+  is the number of pieces in earlier parts; ``num_splits`` is the prefix sum
+  (length ``B + 1``) of the number of pieces of each sequence.
 
 No floating point anywhere.
 """
@@ -53,68 +56,64 @@ def num_parts(rows_per_kv: int, h_kv: int, num_sms: int) -> int:
     return max(1, num_sms // (h_kv * num_row_blocks(rows_per_kv)))
 
 
-def get_metadata(seqlens, rows_per_kv: int, h_kv: int, num_sms: int):
-    """Return ``(tile_md, num_splits)`` as lists of Python ints.
+def _pages(seqlens):
+    return [(int(L) + PAGE - 1) // PAGE if int(L) > 0 else 0 for L in seqlens]
 
-    ``tile_md`` has ``G`` rows of 8 words; ``num_splits`` has ``B + 1``
-    entries.
-    """
+
+def get_metadata(seqlens, rows_per_kv: int, h_kv: int, num_sms: int):
+    """Return ``(tile_md, num_splits)`` as lists of Python ints."""
     C = SPLIT_OVERHEAD_PAGES
-    lens = [int(x) for x in seqlens]
-    B = len(lens)
+    n = _pages(seqlens)
+    B = len(n)
     G = num_parts(rows_per_kv, h_kv, num_sms)
-    n = [(L + PAGE - 1) // PAGE if L > 0 else 0 for L in lens]
-    total = sum(nb + C for nb in n if nb > 0)
-    W = (total + G - 1) // G + C
+    start = []          # P_b
+    acc = 0
+    for nb in n:
+        start.append(acc)
+        acc += nb + C if nb > 0 else 0
+    total = acc
+    W = max(1, (total + G - 1) // G)
+
+    def part_of(unit):
+        return min(unit // W, G - 1)
+
+    # every page, in order, to its part
+    owner = {}
+    for b in range(B):
+        for j in range(n[b]):
+            owner[(b, j)] = part_of(start[b] + C + j)
+
+    def pos(U):
+        for b in range(B):
+            if n[b] > 0 and start[b] + n[b] + C > U:
+                return (b, max(0, U - start[b] - C))
+        return (B, 0)
 
     tile_md = []
-    pieces_of = [0] * B
-    b, page, piece = 0, 0, 0
+    first = 0
     for p in range(G):
-        begin_b, begin_page, first_piece = b, page, piece
-        if p == G - 1:
-            while b < B:
-                if n[b] > page:
-                    pieces_of[b] += 1
-                    piece += 1
-                b, page = b + 1, 0
-        else:
-            remaining = W
-            while b < B:
-                if n[b] == 0:
-                    b, page = b + 1, 0
-                    continue
-                rest = n[b] - page
-                if rest + C <= remaining:
-                    remaining -= rest + C
-                    pieces_of[b] += 1
-                    piece += 1
-                    b, page = b + 1, 0
-                else:
-                    take = remaining - C
-                    if take >= 1:
-                        page += take
-                        pieces_of[b] += 1
-                        piece += 1
-                    break
-        tile_md.append([begin_b, begin_page, b, page, first_piece, piece - first_piece, 0, 0])
+        begin = pos(p * W)
+        end = pos((p + 1) * W) if p < G - 1 else (B, 0)
+        pieces = sorted({b for (b, j), q in owner.items() if q == p})
+        tile_md.append([begin[0], begin[1], end[0], end[1], first, len(pieces), 0, 0])
+        first += len(pieces)
 
     num_splits = [0]
     for b in range(B):
-        num_splits.append(num_splits[-1] + pieces_of[b])
+        parts = {owner[(b, j)] for j in range(n[b])}
+        num_splits.append(num_splits[-1] + len(parts))
     return tile_md, num_splits
 
 
 def part_segments(md_row, seqlens):
     """The (sequence, page_lo, page_hi) pieces a part covers, in order."""
     begin_b, begin_page, end_b, end_page = md_row[:4]
+    n = _pages(seqlens)
     out = []
     b = begin_b
-    while b < len(seqlens) and (b < end_b or (b == end_b and end_page > 0)):
-        L = int(seqlens[b])
-        nb = (L + PAGE - 1) // PAGE if L > 0 else 0
+    while b < len(n) and (b < end_b or (b == end_b and end_page > 0)):
         lo = begin_page if b == begin_b else 0
-        hi = end_page if b == end_b else nb
+        hi = end_page if b == end_b else n[b]
         if hi > lo:
             out.append((b, lo, hi))
         b += 1

@@ -187,3 +187,18 @@ def test_host_side_argument_errors():
                              workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
     with pytest.raises(ValueError):           # wrong dtype is caught before the library
         binding.decode_paged(q.float(), k, bt, sl, 512, md, ns)
+
+
+# ---------------------------------------------------------------- the two decode kernels
+
+@pytest.mark.parametrize("shape", [(1, 128, False), (2, 64, True), (1, 256, False), (3, 32, True)])
+def test_pair_and_single_cta_kernels_both_match_oracle(shape):
+    """More than 64 rows per KV head run on CTA pairs (2-SM MMAs); debug flag 4
+    forces one CTA per 64-row block.  Both must match the oracle."""
+    s_q, h_q, causal = shape
+    w = inputs.build(f"pair{s_q}x{h_q}", [1, 63, 64, 65, 129, 640, 1000], s_q=s_q, h_q=h_q, causal=causal, seed=41)
+    o_ref, l_ref = oracle(w)
+    for flags in (0, 4):
+        for sms in (148, 6):
+            out, lse, _, _ = run_gpu(w, num_sms=sms, debug_flags=flags)
+            compare(w, out, lse, o_ref, l_ref, what=f"s_q={s_q} h_q={h_q} flags={flags} sms={sms}")

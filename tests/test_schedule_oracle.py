@@ -26,29 +26,29 @@ def check_invariants(seqlens, rows_per_kv, h_kv, num_sms):
     C = sch.SPLIT_OVERHEAD_PAGES
     n = [(L + 63) // 64 for L in seqlens]
     total = sum(x + C for x in n if x > 0)
-    W = (total + G - 1) // G + C
+    W = max(1, (total + G - 1) // G)
     assert len(md) == G and len(ns) == B + 1 and ns[0] == 0
     covered = {}
     pieces_seen = [0] * B
     prev_end = (0, 0)
     piece = 0
     for p, row in enumerate(md):
-        assert (row[0], row[1]) == prev_end            # contiguous, ordered
+        if p > 0:
+            assert (row[0], row[1]) == prev_end        # contiguous, ordered
         assert (row[2], row[3]) >= (row[0], row[1])
         prev_end = (row[2], row[3])
         assert row[4] == piece
         segs = sch.part_segments(row, seqlens)
         assert row[5] == len(segs)
-        load = 0
+        pages = 0
         for (b, lo, hi) in segs:
             assert 0 <= lo < hi <= n[b]
             for pg in range(lo, hi):
                 assert (b, pg) not in covered
                 covered[(b, pg)] = p
             pieces_seen[b] += 1
-            load += hi - lo + C
-        if p < G - 1:
-            assert load <= W
+            pages += hi - lo
+        assert pages <= W                                # no part holds more than its units
         piece += len(segs)
     assert prev_end == (B, 0)
     assert set(covered) == {(b, pg) for b in range(B) for pg in range(n[b])}
@@ -91,13 +91,11 @@ def test_long_sequences_get_split():
     assert G == 74
     assert ns[-1] > 8                     # most sequences must be cut
     C = sch.SPLIT_OVERHEAD_PAGES
-    W = (sum(1024 + C for _ in lens) + G - 1) // G + C
-    loads = [sum(hi - lo + C for (_, lo, hi) in sch.part_segments(r, lens)) for r in md]
-    # a part that is not the last and did not run out of work closes only when
-    # fewer than C+1 units of capacity are left
+    W = (sum(1024 + C for _ in lens) + G - 1) // G
+    pages = [sum(hi - lo for (_, lo, hi) in sch.part_segments(r, lens)) for r in md]
+    # every part but the last owns W units, of which at most C are overhead
     for p in range(G - 1):
-        if md[p][2] < len(lens):
-            assert W - C <= loads[p] <= W
+        assert W - C <= pages[p] <= W
 
 
 def test_row_block_rule():
