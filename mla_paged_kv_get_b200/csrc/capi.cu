@@ -223,8 +223,53 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   const int row_blocks = (R + n - 1) / n;
   // 65..128+ rows per KV head: CTA pairs with 2-SM MMAs; otherwise one CTA per row block
   const bool use_pair = R > 64 && !(debug_flags & 4);
-  const cudaError_t le = use_pair ? mla::launch_decode_pair(tm_k, tm_q, a, row_blocks, s)
-                                  : mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s);
+  cudaError_t le;
+  if (use_pair) {
+    mla::PairMaps maps;
+    const cuuint64_t tokens = static_cast<cuuint64_t>(num_pages) * MLA_PAGE_SIZE;
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(h_kv) * MLA_HEAD_DIM * 2;   // one token, all heads
+    {
+      // page chunks: (64 cols, tokens, 9 chunks, heads), box = 3 chunks of 64 tokens (24 KB)
+      const cuuint64_t dims[4] = {64, tokens, 9, static_cast<cuuint64_t>(h_kv)};
+      const cuuint64_t strides[3] = {row_bytes, 128, MLA_HEAD_DIM * 2ull};
+      const cuuint32_t box[4] = {64, 64, 3, 1};
+      const cuuint32_t estr[4] = {1, 1, 1, 1};
+      if (encode(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache_d), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    }
+    for (int rank = 0; rank < 2; ++rank) {
+      // dv quarter of rank r: columns 256 h + 128 r + 64 sub + c -> (64 cols, tokens, 2 sub, 2 halves, heads)
+      const cuuint64_t dims[5] = {64, tokens, 2, 2, static_cast<cuuint64_t>(h_kv)};
+      const cuuint64_t strides[4] = {row_bytes, 128, 512, MLA_HEAD_DIM * 2ull};
+      const cuuint32_t box[5] = {64, 64, 2, 2, 1};
+      const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+      void* base = static_cast<char*>(const_cast<void*>(k_cache_d)) + 256 * rank;
+      if (encode(&maps.v[rank], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    }
+    {
+      // q rows: (64 cols, hg, h_kv, batch*s_q, 9 chunks), box = 64 rows x all 9 chunks (72 KB)
+      const int bh = hg < 64 ? hg : 64;
+      const int bs = 64 / bh;
+      const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(hg), static_cast<cuuint64_t>(h_kv),
+                                  static_cast<cuuint64_t>(batch) * s_q, 9};
+      const cuuint64_t strides[4] = {MLA_HEAD_DIM * 2ull, static_cast<cuuint64_t>(hg) * MLA_HEAD_DIM * 2ull,
+                                     static_cast<cuuint64_t>(h_q) * MLA_HEAD_DIM * 2ull, 128};
+      const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(bh), 1, static_cast<cuuint32_t>(bs), 9};
+      const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+      if (encode(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q_d), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    }
+    le = mla::launch_decode_pair(maps, a, row_blocks, s);
+  } else {
+    le = mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s);
+  }
   if (le != cudaSuccess) return MLA_ERR_CUDA;
   if (debug_flags & 2) return MLA_OK;
   if (mla::launch_combine(num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=

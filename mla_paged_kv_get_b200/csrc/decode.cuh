@@ -31,9 +31,16 @@ int decode_smem_bytes(int rows_per_block);
 cudaError_t launch_decode(int rows_per_block, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                           const DecodeArgs& a, int row_blocks, cudaStream_t stream);
 
+// Tensor maps of the pair kernel: the score product's page chunks (24 KB boxes),
+// each CTA rank's dv quarter of a page (32 KB boxes) and the 64 Q rows (72 KB).
+struct PairMaps {
+  CUtensorMap k;
+  CUtensorMap v[2];
+  CUtensorMap q;
+};
+
 int decode_pair_smem_bytes();
-cudaError_t launch_decode_pair(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, int row_blocks,
-                               cudaStream_t stream);
+cudaError_t launch_decode_pair(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream);
 
 cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
                            __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,

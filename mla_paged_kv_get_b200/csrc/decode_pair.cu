@@ -9,16 +9,21 @@
 //     each CTA loads one.  So every cache byte of the score product crosses
 //     L2 -> SM exactly once, and each SM reads only half of the B operand.
 //   * O = P.V in two M = 128 x N = 256 products (dv halves); each CTA supplies
-//     128 dv columns of both pages (a second, L2-hit read of half the latent
-//     columns) and receives the full P of its own 64 rows.
+//     128 dv columns of each half for both pages (a second, L2-hit read of a
+//     quarter of the latent columns per page) and the P of its own 64 rows.
+//   * Loads are few and large: a TMA instruction costs about the same whether
+//     it moves 8 KB or 24 KB, so the score product's page arrives as three
+//     24 KB boxes (three 64-column chunks each, one 4-D tensor map), the value
+//     quarter of a page as one 32 KB box (5-D map per CTA rank) and Q as one
+//     72 KB box per sequence.
 //   * TMEM per CTA: O (2 x 128 columns: 64 rows x 512 dv in the pair layout
 //     that puts the second half of N in lanes 64..127) and two S buffers
 //     (64 columns each).  Thread t of warps 0-3 owns TMEM lane t: row
 //     t % 64 and key half (or dv quarter) t / 64, so the softmax of a row is
 //     split between two threads and needs no shuffles.
-//   * Separate load rings for the score product (one 8 KB box per slot) and
-//     for the value product (16 KB per slot), each with its own producer warp,
-//     so value loads for tile t overlap the score product of tile t+1.
+//   * Separate load rings for the score product (24 KB slots) and for the
+//     value product (32 KB slots), each with its own producer warp, so value
+//     loads for tile t overlap the score product of tile t+1.
 //   * The leader CTA (rank 0) issues every MMA; the peer's TMA loads complete
 //     on the leader's barriers (cta_group::2 loads, no multicast), MMA
 //     completions are committed to both CTAs, and the peer's softmax warps
@@ -37,23 +42,26 @@ namespace mla {
 namespace {
 
 constexpr int kRows = 64;              // query rows per CTA
-constexpr int kBox = 8192;             // one TMA box: 64 tokens x 64 bf16 columns
-constexpr int kKSlots = 6;             // score ring: one box per slot
-constexpr int kVSlots = 4;             // value ring: two boxes (128 dv of one page) per slot
+constexpr int kBox = 8192;             // one 64-column chunk of 64 tokens (or rows), bf16
+constexpr int kKSlots = 3;             // score ring: three chunks of this CTA's page per slot
+constexpr int kKSlotBytes = 3 * kBox;
+constexpr int kVSlots = 2;             // value ring: [dv half][2 chunks] of one page per slot
+constexpr int kVSlotBytes = 4 * kBox;
 constexpr int kThreads = 224;          // warps 0-3 softmax, 4 score loads, 5 value loads, 6 MMA
-constexpr int kQBytes = 9 * kBox;      // 64 rows x 576
-constexpr int kPBytes = 2 * kBox;      // P: [key half][64 rows][64 keys] bf16
+constexpr int kQBytes = 9 * kBox;      // 64 rows x 576: [chunk][row][64 cols]
+constexpr int kPBytes = 2 * kBox;      // P: [key half][64 rows][64 keys] bf16 (one buffer)
 constexpr int kOffP = kQBytes;
-constexpr int kOffK = kOffP + 2 * kPBytes;
-constexpr int kOffV = kOffK + kKSlots * kBox;
-constexpr int kOffCtrl = kOffV + kVSlots * 2 * kBox;
-constexpr int kSmemBytes = kOffCtrl + 4096 + 1024;
+constexpr int kOffK = kOffP + kPBytes;
+constexpr int kOffV = kOffK + kKSlots * kKSlotBytes;
+constexpr int kOffCtrl = kOffV + kVSlots * kVSlotBytes;
+constexpr int kSmemBytes = kOffCtrl + 1024 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kColO = 0;               // O half h at column 128 h
 constexpr int kColS = 256;             // S buffer b at column 256 + 64 b
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSoftmaxBar = 1;
+constexpr int kPrefetchTiles = 2;      // cache pages are pulled into L2 this many tiles ahead
 
 struct Ctrl {
   uint64_t k_full[kKSlots], k_empty[kKSlots];
@@ -115,7 +123,7 @@ struct PageWindow {
 // ------------------------------------------------------------------ loads
 // Warp 4: Q at each segment start, then the nine 64-column boxes of this CTA's
 // page of every tile, for the score product.
-__device__ void score_loads(const CUtensorMap* tm_k, const CUtensorMap* tm_q, const DecodeArgs& a, Ctrl& ct,
+__device__ void score_loads(const PairMaps& maps, const DecodeArgs& a, Ctrl& ct,
                             uint8_t* qs, uint8_t* ks, const Ctl& ctl, uint32_t rank, int rb, int g,
                             const int32_t* md, uint32_t leader_q_full, uint32_t leader_k_full0) {
   const int lane = threadIdx.x & 31;
@@ -124,8 +132,6 @@ __device__ void score_loads(const CUtensorMap* tm_k, const CUtensorMap* tm_q, co
   const int q_h0 = hg >= kRows ? r0 % hg : 0;
   const int q_s0 = r0 / hg;
   const bool leader = rank == 0;
-  const bool prefetcher = leader && g == 0;
-  const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
   uint32_t kidx = 0;
   int qloads = 0;
   bool alive = true;
@@ -143,37 +149,24 @@ __device__ void score_loads(const CUtensorMap* tm_k, const CUtensorMap* tm_q, co
     if (qloads > 0 && !wait_uniform(&ct.q_empty, (qloads - 1) & 1)) { alive = false; break; }
     if (lane == 0) {
       if (leader) mbar_arrive_expect_tx(&ct.q_full, 2 * kQBytes);
-      for (int c = 0; c < 9; ++c)
-        tma_load_4d_pair(qs + c * kBox, tm_q, leader_q_full, 64 * c, q_h0, g, s.b * a.s_q + q_s0);
+      tma_load_5d_pair(qs, &maps.q, leader_q_full, 0, q_h0, g, s.b * a.s_q + q_s0, 0);
     }
     ++qloads;
     const int32_t* bt_row = a.block_table + static_cast<size_t>(s.b) * a.max_pages;
     win.reset(bt_row, s.hi, a.num_pages, a.status);
-    auto prefetch_tile = [&](int t) {
-      if (!prefetcher || lane != 0) return;
-      for (int q = 0; q < 2; ++q) {
-        const int pg = s.lo + 2 * t + q;
-        if (pg >= s.hi) break;
-        const int id = __ldg(bt_row + pg);
-        if (id >= 0 && id < a.num_pages) l2_prefetch(a.k_cache + static_cast<size_t>(id) * page_bytes, page_bytes);
-      }
-    };
-    prefetch_tile(0);
-    prefetch_tile(1);
 #pragma unroll 1
     for (int t = 0; t < s.ntiles && alive; ++t) {
       const int pid = win.get(s.lo + 2 * t + static_cast<int>(rank));
-      prefetch_tile(t + 2);
 #pragma unroll 1
-      for (int c = 0; c < 9; ++c) {
+      for (int j = 0; j < 3; ++j) {
         const uint32_t slot = kidx % kKSlots;
         if (kidx >= static_cast<uint32_t>(kKSlots) && !wait_uniform(&ct.k_empty[slot], ((kidx / kKSlots) - 1) & 1)) {
           alive = false;
           break;
         }
         if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&ct.k_full[slot], 2 * kBox);
-          tma_load_3d_pair(ks + slot * kBox, tm_k, leader_k_full0 + slot * 8, 64 * c, g, 64 * pid);
+          if (leader) mbar_arrive_expect_tx(&ct.k_full[slot], 2 * kKSlotBytes);
+          tma_load_4d_pair(ks + slot * kKSlotBytes, &maps.k, leader_k_full0 + slot * 8, 0, 64 * pid, 3 * j, g);
         }
         ++kidx;
       }
@@ -183,8 +176,8 @@ __device__ void score_loads(const CUtensorMap* tm_k, const CUtensorMap* tm_q, co
 }
 
 // Warp 5: for the value product of every tile, this CTA's 128 dv columns of each
-// dv half, for both pages: [page q][dv half h] -> one 16 KB slot [box j][64 tokens][64 cols].
-__device__ void value_loads(const CUtensorMap* tm_k, const DecodeArgs& a, Ctrl& ct, uint8_t* vs, const Ctl& ctl,
+// dv half, page by page: one 32 KB slot [dv half][chunk][64 tokens][64 cols].
+__device__ void value_loads(const PairMaps& maps, const DecodeArgs& a, Ctrl& ct, uint8_t* vs, const Ctl& ctl,
                             uint32_t rank, int g, const int32_t* md, uint32_t leader_v_full0) {
   const int lane = threadIdx.x & 31;
   const bool leader = rank == 0;
@@ -206,20 +199,16 @@ __device__ void value_loads(const CUtensorMap* tm_k, const DecodeArgs& a, Ctrl& 
     for (int t = 0; t < s.ntiles && alive; ++t) {
       const int pid0 = win.get(s.lo + 2 * t), pid1 = win.get(s.lo + 2 * t + 1);
 #pragma unroll 1
-      for (int u = 0; u < 4; ++u) {     // u = 2 h + q
-        const int h = u >> 1, q = u & 1;
+      for (int q = 0; q < 2; ++q) {     // page q of the tile: this CTA's dv quarter of both halves
         const uint32_t slot = vidx % kVSlots;
         if (vidx >= static_cast<uint32_t>(kVSlots) && !wait_uniform(&ct.v_empty[slot], ((vidx / kVSlots) - 1) & 1)) {
           alive = false;
           break;
         }
         if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&ct.v_full[slot], 4 * kBox);
-          const int col = 256 * h + 128 * static_cast<int>(rank);
-          const int pid = q ? pid1 : pid0;
-          uint8_t* dst = vs + slot * 2 * kBox;
-          tma_load_3d_pair(dst, tm_k, leader_v_full0 + slot * 8, col, g, 64 * pid);
-          tma_load_3d_pair(dst + kBox, tm_k, leader_v_full0 + slot * 8, col + 64, g, 64 * pid);
+          if (leader) mbar_arrive_expect_tx(&ct.v_full[slot], 2 * kVSlotBytes);
+          tma_load_5d_pair(vs + slot * kVSlotBytes, &maps.v[rank], leader_v_full0 + slot * 8, 0, 64 * (q ? pid1 : pid0),
+                           0, 0, g);
         }
         ++vidx;
       }
@@ -256,15 +245,18 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
       tc_fence_after();
       const uint32_t d_tmem = tmem + kColS + 64 * sb;
 #pragma unroll 1
-      for (int c = 0; c < 9; ++c) {
+      for (int j = 0; j < 3; ++j) {
         const uint32_t slot = kidx % kKSlots;
         if (!wait_phase(&ct.k_full[slot], (kidx / kKSlots) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc(q_addr + c * kBox + kk * 32, 16, 1024, 2);
-          const uint64_t bd = smem_desc(k_addr + slot * kBox + kk * 32, 16, 1024, 2);
-          umma_bf16_pair(d_tmem, ad, bd, idesc_qk, (c | kk) != 0 ? 1u : 0u);
+        for (int cc = 0; cc < 3; ++cc) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc(q_addr + (3 * j + cc) * kBox + kk * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(k_addr + slot * kKSlotBytes + cc * kBox + kk * 32, 16, 1024, 2);
+            umma_bf16_pair(d_tmem, ad, bd, idesc_qk, (j | cc | kk) != 0 ? 1u : 0u);
+          }
         }
         umma_commit_pair(&ct.k_empty[slot]);
         ++kidx;
@@ -280,18 +272,20 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
       if (!wait_phase_cluster(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
       tc_fence_after();
 #pragma unroll 1
-      for (int u = 0; u < 4; ++u) {       // u = 2 h + q: dv half h, page q of the tile
-        const int h = u >> 1, q = u & 1;
+      for (int q = 0; q < 2; ++q) {       // page q of the tile
         const uint32_t slot = vidx % kVSlots;
         if (!wait_phase(&ct.v_full[slot], (vidx / kVSlots) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          // A = P: 128 rows (64 per CTA) x 16 keys of page q, K-major
-          const uint64_t ad = smem_desc(p_addr + pb * kPBytes + q * kBox + kk * 32, 16, 1024, 2);
-          // B = V: 16 keys x 256 dv (128 per CTA: two boxes 8 KB apart), MN-major
-          const uint64_t bd = smem_desc(v_addr + slot * 2 * kBox + kk * 2048, kBox, 1024, 2);
-          umma_bf16_pair(tmem + kColO + 128 * h, ad, bd, idesc_pv, (t > 0 || q > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {     // dv half
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // A = P: 128 rows (64 per CTA) x 16 keys of page q, K-major
+            const uint64_t ad = smem_desc(p_addr + q * kBox + kk * 32, 16, 1024, 2);
+            // B = V: 16 keys x 256 dv (128 per CTA: two chunks 8 KB apart), MN-major
+            const uint64_t bd = smem_desc(v_addr + slot * kVSlotBytes + h * 2 * kBox + kk * 2048, kBox, 1024, 2);
+            umma_bf16_pair(tmem + kColO + 128 * h, ad, bd, idesc_pv, (t > 0 || q > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit_pair(&ct.v_empty[slot]);
         ++vidx;
@@ -348,12 +342,29 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
     }
     if (!s.ok && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
     float m_run = -INFINITY, lsum = 0.f;
+    // L2 prefetch of this CTA's page kPrefetchTiles ahead: its 576 lines spread over the 128
+    // threads.  The page id is read one tile before it is used so the load latency is hidden.
+    const int32_t* bt_row = a.block_table + static_cast<size_t>(s.b) * a.max_pages;
+    const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
+    auto page_of_tile = [&](int t) -> int {
+      const int pg = s.lo + 2 * t + static_cast<int>(rank);
+      if (t >= s.ntiles || pg >= s.hi) return -1;
+      const int id = __ldg(bt_row + pg);
+      return id >= 0 && id < a.num_pages ? id : -1;
+    };
+    int pf_next = page_of_tile(kPrefetchTiles);
 
 #pragma unroll 1
     for (int t = 0; t < s.ntiles; ++t, ++tg) {
       const int sb = tg & 1;
+      if (pf_next >= 0) {
+        const uint8_t* pg = a.k_cache + static_cast<size_t>(pf_next) * page_bytes;
+        for (int line = tid; line * 128 < static_cast<int>(page_bytes); line += 128) l2_prefetch_line(pg + line * 128);
+      }
+      pf_next = page_of_tile(t + 1 + kPrefetchTiles);
       bool ok = wait_phase(&ct.s_full[sb], (tg >> 1) & 1, ctl);
-      if (ok && tg >= 2) ok = wait_phase(&ct.p_free[sb], ((tg >> 1) - 1) & 1, ctl);   // P buffer sb free
+      // the single P buffer is free once the value product of the previous tile has finished
+      if (ok && tg >= 1) ok = wait_phase(&ct.p_free[(tg - 1) & 1], ((tg - 1) >> 1) & 1, ctl);
       float x[64];
       bool need = false;
       float mloc = -INFINITY;
@@ -370,12 +381,22 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_s_free0 + sb * 8);
-        const int key0 = (s.lo + 2 * t) * 64 + 64 * kh;
+        const int nvis = kmax - ((s.lo + 2 * t) * 64 + 64 * kh);   // visible keys of this half
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (nvis >= 64) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = key0 + j < kmax ? x[j] * a.scale_log2 : -INFINITY;
-          mloc = fmaxf(mloc, x[j]);
+          for (int j = 0; j < 64; ++j) {
+            x[j] *= a.scale_log2;
+            m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            x[j] = j < nvis ? x[j] * a.scale_log2 : -INFINITY;
+            m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+          }
         }
+        mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         need = mloc > m_run + kTau;
       }
       if (!ok) ct.softmax_abort = 1;
@@ -391,8 +412,7 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
         m_run = mn;
         lsum *= alpha;
         if (t > 0) {
-          const bool okr = wait_phase(&ct.p_free[(tg - 1) & 1], ((tg - 1) >> 1) & 1, ctl);
-          if (!uniform_ok(okr)) return;
+          // the value product of tile tg-1 has finished (waited above): rescale O in TMEM
           tc_fence_after();
 #pragma unroll 1
           for (int c16 = 0; c16 < 16; ++c16) {     // this lane's 256 O columns (both dv halves)
@@ -409,21 +429,23 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
         named_sync(kSoftmaxBar, 128);              // red[] is reused by the next tile
       }
 
-      // P row slice: 64 keys of this thread's half, 128 bytes, 128-byte swizzle
-      uint8_t* prow = ps + (tg & 1) * kPBytes + kh * kBox + r * 128;
+      // P row slice: 64 keys of this thread's half, 128 bytes, 128-byte swizzle.
+      // exp2(-inf - m) = 0 for masked keys; m_run is finite once a key was seen.
+      uint8_t* prow = ps + kh * kBox + r * 128;
+      const float mneg = m_run == -INFINITY ? 0.f : -m_run;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = 8 * c8 + 2 * i;
-          const float p0 = x[j] == -INFINITY ? 0.f : ex2(x[j] - m_run);
-          const float p1 = x[j + 1] == -INFINITY ? 0.f : ex2(x[j + 1] - m_run);
-          w[i] = pack_bf16(p0, p1);
-          lsum += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+          w[i] = pack_bf16(ex2(x[j] + mneg), ex2(x[j + 1] + mneg));
+          l4[i] += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
         }
         *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      lsum += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       fence_async_shared();
       tc_fence_before();
       __syncwarp();
@@ -495,8 +517,7 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                       const DecodeArgs a) {
+mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* qs = smem;
@@ -540,8 +561,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     tmem_relinquish_pair();
   }
   if (warp == 4 && (threadIdx.x & 31) == 0) {
-    tma_prefetch_map(&tm_k);
-    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&maps.k);
+    tma_prefetch_map(&maps.q);
+    tma_prefetch_map(&maps.v[0]);
+    tma_prefetch_map(&maps.v[1]);
   }
   tc_fence_before();
   __syncthreads();
@@ -561,9 +584,9 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
   if (warp < 4) {
     softmax_rows(a, ct, ps, tmem, ctl, rank, rb, g, md, L_s_free0, L_p_full0, L_o_free);
   } else if (warp == 4) {
-    score_loads(&tm_k, &tm_q, a, ct, qs, ks, ctl, rank, rb, g, md, L_q_full, L_k_full0);
+    score_loads(maps, a, ct, qs, ks, ctl, rank, rb, g, md, L_q_full, L_k_full0);
   } else if (warp == 5) {
-    value_loads(&tm_k, a, ct, vs, ctl, rank, g, md, L_v_full0);
+    value_loads(maps, a, ct, vs, ctl, rank, g, md, L_v_full0);
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {
     clean = mma_issue(a, ct, qs, ps, ks, vs, tmem, ctl, md);
     if (!clean) {
@@ -585,8 +608,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 
 int decode_pair_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_decode_pair(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, int row_blocks,
-                               cudaStream_t stream) {
+cudaError_t launch_decode_pair(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream) {
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -598,7 +620,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_k, const CUtensorMap& tm_q,
   }
   const int pairs = (row_blocks + 1) / 2;
   const dim3 grid(2 * pairs, a.h_kv, a.num_parts);
-  mla_decode_pair_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, a);
+  mla_decode_pair_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
   return cudaGetLastError();
 }
 
