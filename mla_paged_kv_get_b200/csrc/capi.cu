@@ -163,34 +163,34 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   EncodeTiledFn encode = encode_fn();
   if (encode == nullptr) return MLA_ERR_CUDA;
 
-  // cache: [num_pages * 64 tokens][h_kv][576] -> dims (576, h_kv, tokens), box 64 cols x 1 head x 64 tokens
-  CUtensorMap tm_k, tm_q;
-  {
-    const cuuint64_t dims[3] = {MLA_HEAD_DIM, static_cast<cuuint64_t>(h_kv),
-                                static_cast<cuuint64_t>(num_pages) * MLA_PAGE_SIZE};
-    const cuuint64_t strides[2] = {MLA_HEAD_DIM * 2ull, static_cast<cuuint64_t>(h_kv) * MLA_HEAD_DIM * 2ull};
-    const cuuint32_t box[3] = {64, 1, 64};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    if (encode(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k_cache_d), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return MLA_ERR_CUDA;
-  }
-  // q: [batch * s_q][h_kv][hg][576] -> dims (576, hg, h_kv, batch*s_q); box 64 cols x bh heads x 1 x bs tokens
-  {
-    const int bh = hg < n ? hg : n;
-    const int bs = n / bh;
-    const cuuint64_t dims[4] = {MLA_HEAD_DIM, static_cast<cuuint64_t>(hg), static_cast<cuuint64_t>(h_kv),
-                                static_cast<cuuint64_t>(batch) * s_q};
-    const cuuint64_t strides[3] = {MLA_HEAD_DIM * 2ull, static_cast<cuuint64_t>(hg) * MLA_HEAD_DIM * 2ull,
-                                   static_cast<cuuint64_t>(h_q) * MLA_HEAD_DIM * 2ull};
-    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(bh), 1, static_cast<cuuint32_t>(bs)};
+  const cuuint64_t tokens = static_cast<cuuint64_t>(num_pages) * MLA_PAGE_SIZE;
+  const cuuint64_t token_bytes = static_cast<cuuint64_t>(h_kv) * MLA_HEAD_DIM * 2;   // one token, all heads
+  // Cache pages as (64 cols, tokens, 9 chunks, heads): a box of `chunks` 64-column chunks of 64 tokens
+  // lands in shared memory as [chunk][token][64 cols], the 128-byte swizzled K-major tile layout.
+  auto page_map = [&](CUtensorMap* m, int chunks) -> bool {
+    const cuuint64_t dims[4] = {64, tokens, 9, static_cast<cuuint64_t>(h_kv)};
+    const cuuint64_t strides[3] = {token_bytes, 128, MLA_HEAD_DIM * 2ull};
+    const cuuint32_t box[4] = {64, 64, static_cast<cuuint32_t>(chunks), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q_d), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return MLA_ERR_CUDA;
-  }
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache_d), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  // Q rows as (64 cols, hg, h_kv, batch*s_q, 9 chunks): a box of `rows` query rows and all nine chunks
+  // lands as [chunk][row][64 cols].
+  auto q_map = [&](CUtensorMap* m, int rows) -> bool {
+    const int bh = hg < rows ? hg : rows;
+    const int bs = rows / bh;
+    const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(hg), static_cast<cuuint64_t>(h_kv),
+                                static_cast<cuuint64_t>(batch) * s_q, 9};
+    const cuuint64_t strides[4] = {MLA_HEAD_DIM * 2ull, static_cast<cuuint64_t>(hg) * MLA_HEAD_DIM * 2ull,
+                                   static_cast<cuuint64_t>(h_q) * MLA_HEAD_DIM * 2ull, 128};
+    const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(bh), 1, static_cast<cuuint32_t>(bs), 9};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q_d), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
 
   mla::DecodeArgs a;
   a.k_cache = static_cast<const uint8_t*>(k_cache_d);
@@ -226,23 +226,11 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   cudaError_t le;
   if (use_pair) {
     mla::PairMaps maps;
-    const cuuint64_t tokens = static_cast<cuuint64_t>(num_pages) * MLA_PAGE_SIZE;
-    const cuuint64_t row_bytes = static_cast<cuuint64_t>(h_kv) * MLA_HEAD_DIM * 2;   // one token, all heads
-    {
-      // page chunks: (64 cols, tokens, 9 chunks, heads), box = 3 chunks of 64 tokens (24 KB)
-      const cuuint64_t dims[4] = {64, tokens, 9, static_cast<cuuint64_t>(h_kv)};
-      const cuuint64_t strides[3] = {row_bytes, 128, MLA_HEAD_DIM * 2ull};
-      const cuuint32_t box[4] = {64, 64, 3, 1};
-      const cuuint32_t estr[4] = {1, 1, 1, 1};
-      if (encode(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache_d), dims, strides, box, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return MLA_ERR_CUDA;
-    }
+    if (!page_map(&maps.k, 3)) return MLA_ERR_CUDA;
     for (int rank = 0; rank < 2; ++rank) {
       // dv quarter of rank r: columns 256 h + 128 r + 64 sub + c -> (64 cols, tokens, 2 sub, 2 halves, heads)
       const cuuint64_t dims[5] = {64, tokens, 2, 2, static_cast<cuuint64_t>(h_kv)};
-      const cuuint64_t strides[4] = {row_bytes, 128, 512, MLA_HEAD_DIM * 2ull};
+      const cuuint64_t strides[4] = {token_bytes, 128, 512, MLA_HEAD_DIM * 2ull};
       const cuuint32_t box[5] = {64, 64, 2, 2, 1};
       const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
       void* base = static_cast<char*>(const_cast<void*>(k_cache_d)) + 256 * rank;
@@ -251,23 +239,11 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return MLA_ERR_CUDA;
     }
-    {
-      // q rows: (64 cols, hg, h_kv, batch*s_q, 9 chunks), box = 64 rows x all 9 chunks (72 KB)
-      const int bh = hg < 64 ? hg : 64;
-      const int bs = 64 / bh;
-      const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(hg), static_cast<cuuint64_t>(h_kv),
-                                  static_cast<cuuint64_t>(batch) * s_q, 9};
-      const cuuint64_t strides[4] = {MLA_HEAD_DIM * 2ull, static_cast<cuuint64_t>(hg) * MLA_HEAD_DIM * 2ull,
-                                     static_cast<cuuint64_t>(h_q) * MLA_HEAD_DIM * 2ull, 128};
-      const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(bh), 1, static_cast<cuuint32_t>(bs), 9};
-      const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-      if (encode(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q_d), dims, strides, box, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return MLA_ERR_CUDA;
-    }
+    if (!q_map(&maps.q, 64)) return MLA_ERR_CUDA;
     le = mla::launch_decode_pair(maps, a, row_blocks, s);
   } else {
+    CUtensorMap tm_k, tm_q;
+    if (!page_map(&tm_k, 1) || !q_map(&tm_q, n)) return MLA_ERR_CUDA;
     le = mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s);
   }
   if (le != cudaSuccess) return MLA_ERR_CUDA;

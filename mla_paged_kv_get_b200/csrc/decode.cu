@@ -47,13 +47,18 @@ namespace {
 constexpr int kKeys = 128;          // keys per tile (two pages)
 constexpr int kSlotBytes = 16384;   // one ring slot: two 64 x 64 boxes
 constexpr int kBoxBytes = 8192;     // one TMA box: 64 tokens x 64 bf16 columns
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 4;
 constexpr float kTau = 8.0f;        // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSoftmaxBar = 1;      // named barrier of warps 0-3
 
 template <int N>
 struct Cfg {
+  // TMA issue is the bottleneck of 8 KB boxes (one warp moves ~28 GB/s): several producer
+  // warps issue interleaved loads.  N = 64 keeps two so that 256 threads keep 255 registers.
+  static constexpr int kProducers = N == 64 ? 2 : 4;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + kProducers + 1);
+  static constexpr int kMmaWarp = kSoftmaxWarps + kProducers;
   static constexpr int kSlots = N == 64 ? 8 : (N == 32 ? 10 : 12);
   static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
   static constexpr int kQBytes = N * 128 * 9;          // 9 chunks of [N rows][64 cols]
@@ -103,11 +108,14 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// ------------------------------------------------------------------ producer
+// ------------------------------------------------------------------ producers (warps 4 ..)
+// The slot-load sequence of a segment is fixed: Q, QK(0), then QK(t), PV(t-1) for t >= 1, then
+// PV(T-1); QK(t) is nine slots (one 64-column chunk of both pages), PV(t) eight (128 dv columns of
+// one page).  Producer warp w issues the loads whose index is w modulo the number of producers.
 template <int N>
 __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, const DecodeArgs& a,
                               Ctrl& ct, uint8_t* slots, uint8_t* qs, const Ctl& ctl, int rb, int g,
-                              const int32_t* md) {
+                              const int32_t* md, int pw) {
   using C = Cfg<N>;
   const int lane = threadIdx.x & 31;
   const int hg = a.hg;
@@ -133,12 +141,12 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
 
   while (alive && it.next(a, s)) {
     if (s.ntiles == 0) continue;
-    if (qloads > 0 && !wait_uniform(&ct.q_empty, (qloads - 1) & 1)) { alive = false; break; }
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&ct.q_full, C::kQBytes);
-#pragma unroll 1
-      for (int c = 0; c < 9; ++c)
-        tma_load_4d(qs + c * N * 128, tm_q, &ct.q_full, 64 * c, q_h0, g, s.b * a.s_q + q_s0);
+    if (pw == 0) {
+      if (qloads > 0 && !wait_uniform(&ct.q_empty, (qloads - 1) & 1)) { alive = false; break; }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&ct.q_full, C::kQBytes);
+        tma_load_5d(qs, tm_q, &ct.q_full, 0, q_h0, g, s.b * a.s_q + q_s0, 0);
+      }
     }
     ++qloads;
 
@@ -161,67 +169,39 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
       return v;
     };
 
-    auto acquire_slot = [&](uint32_t& slot) -> bool {
-      slot = load_idx % C::kSlots;
-      if (load_idx >= static_cast<uint32_t>(C::kSlots))
-        return wait_uniform(&ct.empty[slot], ((load_idx / C::kSlots) - 1) & 1);
+    // one slot: two 8 KB boxes; returns false when the CTA is aborting
+    auto issue = [&](int chunk0, int chunk1, int pid0, int pid1) -> bool {
+      const uint32_t idx = load_idx++;
+      if (static_cast<int>(idx % C::kProducers) != pw) return true;
+      const uint32_t slot = idx % C::kSlots;
+      if (idx >= static_cast<uint32_t>(C::kSlots) && !wait_uniform(&ct.empty[slot], ((idx / C::kSlots) - 1) & 1))
+        return false;
+      if (lane == 0) {
+        uint8_t* dst = slots + slot * kSlotBytes;
+        mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
+        tma_load_4d(dst, tm_k, &ct.full[slot], 0, 64 * pid0, chunk0, g);
+        tma_load_4d(dst + kBoxBytes, tm_k, &ct.full[slot], 0, 64 * pid1, chunk1, g);
+      }
       return true;
     };
-
-    // pages two tiles ahead are pulled into L2 (one CTA of the row blocks and heads does it)
-    const bool prefetcher = rb == 0 && g == 0;
-    const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
-    auto prefetch_tile = [&](int t) {
-      if (!prefetcher || lane != 0) return;
-      for (int q = 0; q < 2; ++q) {
-        const int pg = s.lo + 2 * t + q;
-        if (pg >= s.hi) break;
-        const int id = __ldg(bt_row + pg);
-        if (id >= 0 && id < a.num_pages) l2_prefetch(a.k_cache + static_cast<size_t>(id) * page_bytes, page_bytes);
-      }
-    };
-
     auto issue_qk = [&](int t) -> bool {
+      // [page][64 tokens][64 cols]: the 128 keys of the tile contiguous, one column chunk
       const int pid0 = page_id(s.lo + 2 * t), pid1 = page_id(s.lo + 2 * t + 1);
-      prefetch_tile(t + 2);
-#pragma unroll 1
-      for (int c = 0; c < 9; ++c) {
-        uint32_t slot;
-        if (!acquire_slot(slot)) return false;
-        if (lane == 0) {
-          // [page][64 tokens][64 cols]: the 128 keys of the tile contiguous, one column chunk
-          uint8_t* dst = slots + slot * kSlotBytes;
-          mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
-          tma_load_3d(dst, tm_k, &ct.full[slot], 64 * c, g, 64 * pid0);
-          tma_load_3d(dst + kBoxBytes, tm_k, &ct.full[slot], 64 * c, g, 64 * pid1);
-        }
-        ++load_idx;
-      }
+      for (int c = 0; c < 9; ++c)
+        if (!issue(c, c, pid0, pid1)) return false;
       return true;
     };
-
     auto issue_pv = [&](int t) -> bool {
+      // [chunk j][64 tokens][64 cols] of one page: 128 dv columns of 64 keys
       const int pid0 = page_id(s.lo + 2 * t), pid1 = page_id(s.lo + 2 * t + 1);
-#pragma unroll 1
       for (int u = 0; u < 8; ++u) {
-        uint32_t slot;
-        if (!acquire_slot(slot)) return false;
-        if (lane == 0) {
-          // [chunk j][64 tokens][64 cols] of one page: 128 dv columns of 64 keys
-          uint8_t* dst = slots + slot * kSlotBytes;
-          const int pid = (u & 1) ? pid1 : pid0;
-          const int col = 128 * (u >> 1);
-          mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
-          tma_load_3d(dst, tm_k, &ct.full[slot], col, g, 64 * pid);
-          tma_load_3d(dst + kBoxBytes, tm_k, &ct.full[slot], col + 64, g, 64 * pid);
-        }
-        ++load_idx;
+        const int pid = (u & 1) ? pid1 : pid0;
+        const int c = 2 * (u >> 1);
+        if (!issue(c, c + 1, pid, pid)) return false;
       }
       return true;
     };
 
-    prefetch_tile(0);
-    prefetch_tile(1);
     if (!issue_qk(0)) { alive = false; break; }
 #pragma unroll 1
     for (int t = 1; t < s.ntiles && alive; ++t) {
@@ -232,12 +212,12 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
 
   if (!alive && lane == 0) {
     // unwind: let every TMA load this warp issued land before the CTA exits
-    const uint32_t n = load_idx < static_cast<uint32_t>(C::kSlots) ? load_idx : C::kSlots;
-    for (uint32_t i = 0; i < n; ++i) {
+    for (uint32_t i = 0; i < static_cast<uint32_t>(C::kSlots) && i < load_idx; ++i) {
       const uint32_t li = load_idx - 1 - i;
-      drain_phase(&ct.full[li % C::kSlots], (li / C::kSlots) & 1, 1000000000ull);
+      if (static_cast<int>(li % C::kProducers) == pw)
+        drain_phase(&ct.full[li % C::kSlots], (li / C::kSlots) & 1, 1000000000ull);
     }
-    if (qloads > 0) drain_phase(&ct.q_full, (qloads - 1) & 1, 1000000000ull);
+    if (pw == 0 && qloads > 0) drain_phase(&ct.q_full, (qloads - 1) & 1, 1000000000ull);
   }
   __syncwarp();
 }
@@ -571,7 +551,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
 }
 
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<N>::kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const DecodeArgs a) {
   using C = Cfg<N>;
@@ -606,11 +586,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     ct.softmax_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == C::kMmaWarp) {
     tmem_alloc(&ct.tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && (threadIdx.x & 31) == 0) {
+  if (warp == kSoftmaxWarps && (threadIdx.x & 31) == 0) {
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_q);
   }
@@ -620,17 +600,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const uint32_t tmem = ct.tmem_base;
   const Ctl ctl{&ct.abort_flag, a.status, a.timeout_ns};
 
-  if (warp < 4) {
+  if (warp < kSoftmaxWarps) {
     softmax_role<N>(a, ct, ps, tmem, ctl, rb, g, md);
-  } else if (warp == 4) {
-    producer_role<N>(&tm_k, &tm_q, a, ct, slots, qs, ctl, rb, g, md);
+  } else if (warp < C::kMmaWarp) {
+    producer_role<N>(&tm_k, &tm_q, a, ct, slots, qs, ctl, rb, g, md, warp - kSoftmaxWarps);
   } else {
     mma_role<N>(a, ct, slots, qs, ps, tmem, ctl, md);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -659,7 +639,7 @@ static cudaError_t launch_n(const CUtensorMap& tm_k, const CUtensorMap& tm_q, co
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  mla_decode_kernel<N><<<grid, kThreads, Cfg<N>::kSmemBytes, stream>>>(tm_k, tm_q, a);
+  mla_decode_kernel<N><<<grid, Cfg<N>::kThreads, Cfg<N>::kSmemBytes, stream>>>(tm_k, tm_q, a);
   return cudaGetLastError();
 }
 

@@ -61,7 +61,6 @@ constexpr int kColS = 256;             // S buffer b at column 256 + 64 b
 constexpr float kTau = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSoftmaxBar = 1;
-constexpr int kPrefetchTiles = 2;      // cache pages are pulled into L2 this many tiles ahead
 
 struct Ctrl {
   uint64_t k_full[kKSlots], k_empty[kKSlots];
@@ -342,26 +341,10 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
     }
     if (!s.ok && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
     float m_run = -INFINITY, lsum = 0.f;
-    // L2 prefetch of this CTA's page kPrefetchTiles ahead: its 576 lines spread over the 128
-    // threads.  The page id is read one tile before it is used so the load latency is hidden.
-    const int32_t* bt_row = a.block_table + static_cast<size_t>(s.b) * a.max_pages;
-    const size_t page_bytes = static_cast<size_t>(64) * a.h_kv * 576 * 2;
-    auto page_of_tile = [&](int t) -> int {
-      const int pg = s.lo + 2 * t + static_cast<int>(rank);
-      if (t >= s.ntiles || pg >= s.hi) return -1;
-      const int id = __ldg(bt_row + pg);
-      return id >= 0 && id < a.num_pages ? id : -1;
-    };
-    int pf_next = page_of_tile(kPrefetchTiles);
 
 #pragma unroll 1
     for (int t = 0; t < s.ntiles; ++t, ++tg) {
       const int sb = tg & 1;
-      if (pf_next >= 0) {
-        const uint8_t* pg = a.k_cache + static_cast<size_t>(pf_next) * page_bytes;
-        for (int line = tid; line * 128 < static_cast<int>(page_bytes); line += 128) l2_prefetch_line(pg + line * 128);
-      }
-      pf_next = page_of_tile(t + 1 + kPrefetchTiles);
       bool ok = wait_phase(&ct.s_full[sb], (tg >> 1) & 1, ctl);
       // the single P buffer is free once the value product of the previous tile has finished
       if (ok && tg >= 1) ok = wait_phase(&ct.p_free[(tg - 1) & 1], ((tg - 1) >> 1) & 1, ctl);
