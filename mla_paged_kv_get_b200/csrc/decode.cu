@@ -17,13 +17,15 @@
 //     O^T (4N columns) and two S^T buffers (2N columns).
 //   * Warp roles: warps 0-3 own TMEM lanes 0-127 (one key per thread for S,
 //     one dv value per thread for O) and do masking, the online softmax and
-//     the epilogue; warp 4 issues TMA loads; warp 5 (one thread) issues MMAs.
+//     the epilogue; the next warps issue TMA loads; one thread of the last
+//     warp but one issues the score MMAs, one of the last warp the value MMAs.
 //   * The cache is read through the page table by TMA (128-byte swizzle,
-//     64 x 64 boxes) into a ring of 32 KB slots on mbarriers.  A tile is
-//     streamed twice: five slots for the score product (column chunks of 128)
-//     and four slots for the value product (the first 512 columns again; the
-//     second read is an L2 hit).  This keeps the ring independent of the tile
-//     size, which does not fit in shared memory next to Q.
+//     64 x 64 boxes, two per 16 KB ring slot) on mbarriers.  A tile is
+//     streamed twice: nine slots for the score product (one 64-column chunk
+//     of both pages each) and eight for the value product (128 dv columns of
+//     one page each; the second read is an L2 hit).  This keeps the ring
+//     independent of the tile size, which does not fit in shared memory next
+//     to Q.
 //   * Online softmax in log2 units with a lazy rescale: the running max moves
 //     only when a score exceeds it by more than TAU = 8 (a factor 256); the
 //     final normalisation uses the same running max, so the result is exact
@@ -57,9 +59,17 @@ struct Cfg {
   // TMA issue is the bottleneck of 8 KB boxes (one warp moves ~28 GB/s): several producer
   // warps issue interleaved loads.  N = 64 keeps two so that 256 threads keep 255 registers.
   static constexpr int kProducers = N == 64 ? 2 : 4;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + kProducers + 1);
-  static constexpr int kMmaWarp = kSoftmaxWarps + kProducers;
-  static constexpr int kSlots = N == 64 ? 8 : (N == 32 ? 10 : 12);
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + kProducers + 2);
+  static constexpr int kMmaWarp = kSoftmaxWarps + kProducers;   // score-product issuer; owns TMEM
+  static constexpr int kPvWarp = kMmaWarp + 1;                   // value-product issuer
+  // Two rings, one per MMA issuer: score-product chunks (from HBM) and value-product chunks (the
+  // same pages again, L2 hits).  A phase-parity wait is only sound when the waiter is at most
+  // one phase ahead, so each ring has one consumer that takes it in order, and each slot one
+  // producer warp (ring index modulo the producer count, ring sizes multiples of it).
+  static constexpr int kSlotsQk = N == 16 ? 8 : 4;
+  static constexpr int kSlotsPv = 4;
+  static constexpr int kSlots = kSlotsQk + kSlotsPv;
+  static_assert(kSlotsQk % kProducers == 0 && kSlotsPv % kProducers == 0, "slot ownership");
   static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
   static constexpr int kQBytes = N * 128 * 9;          // 9 chunks of [N rows][64 cols]
   static constexpr int kPBytes = kKeys * N * 2;        // P^T: [128 keys][N rows] bf16
@@ -79,7 +89,7 @@ struct Ctrl {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
-  uint64_t o_free, never, drain;
+  uint64_t o_free, never, drain[2];
   uint32_t tmem_base;
   int abort_flag;         // any role gave up
   int softmax_abort;      // written only by warps 0-3, read after their barrier
@@ -110,8 +120,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ------------------------------------------------------------------ producers (warps 4 ..)
 // The slot-load sequence of a segment is fixed: Q, QK(0), then QK(t), PV(t-1) for t >= 1, then
-// PV(T-1); QK(t) is nine slots (one 64-column chunk of both pages), PV(t) eight (128 dv columns of
-// one page).  Producer warp w issues the loads whose index is w modulo the number of producers.
+// PV(T-1); QK(t) is nine loads (one 64-column chunk of both pages), PV(t) eight (128 dv columns of
+// one page).  QK loads go to the score ring, PV loads to the value ring.  Producer warp w issues
+// the loads whose index in their ring is w modulo the number of producers, so it owns fixed
+// slots and waits only for the consumption of its own earlier loads.
 template <int N>
 __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, const DecodeArgs& a,
                               Ctrl& ct, uint8_t* slots, uint8_t* qs, const Ctl& ctl, int rb, int g,
@@ -125,7 +137,8 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
   const int q_s0 = r0 / hg;
   const int oob_page = a.num_pages;   // page coordinate past the cache: zero-filled box
 
-  uint32_t load_idx = 0;
+  uint32_t qk_idx = 0, pv_idx = 0;
+  uint32_t mine = 0, mine_parity = 0;   // slots holding a load of this warp, and its phase parity
   int qloads = 0;
   bool alive = true;
   SegIter it;
@@ -170,12 +183,14 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
     };
 
     // one slot: two 8 KB boxes; returns false when the CTA is aborting
-    auto issue = [&](int chunk0, int chunk1, int pid0, int pid1) -> bool {
-      const uint32_t idx = load_idx++;
-      if (static_cast<int>(idx % C::kProducers) != pw) return true;
-      const uint32_t slot = idx % C::kSlots;
-      if (idx >= static_cast<uint32_t>(C::kSlots) && !wait_uniform(&ct.empty[slot], ((idx / C::kSlots) - 1) & 1))
-        return false;
+    auto issue = [&](bool pv, int chunk0, int chunk1, int pid0, int pid1) -> bool {
+      const uint32_t ridx = pv ? pv_idx++ : qk_idx++;
+      if (static_cast<int>(ridx % C::kProducers) != pw) return true;
+      const uint32_t n = pv ? C::kSlotsPv : C::kSlotsQk;
+      const uint32_t slot = (pv ? C::kSlotsQk : 0) + ridx % n;
+      if (ridx >= n && !wait_uniform(&ct.empty[slot], ((ridx / n) - 1) & 1)) return false;
+      mine |= 1u << slot;
+      mine_parity = (mine_parity & ~(1u << slot)) | (((ridx / n) & 1u) << slot);
       if (lane == 0) {
         uint8_t* dst = slots + slot * kSlotBytes;
         mbar_arrive_expect_tx(&ct.full[slot], 2 * kBoxBytes);
@@ -188,7 +203,7 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
       // [page][64 tokens][64 cols]: the 128 keys of the tile contiguous, one column chunk
       const int pid0 = page_id(s.lo + 2 * t), pid1 = page_id(s.lo + 2 * t + 1);
       for (int c = 0; c < 9; ++c)
-        if (!issue(c, c, pid0, pid1)) return false;
+        if (!issue(false, c, c, pid0, pid1)) return false;
       return true;
     };
     auto issue_pv = [&](int t) -> bool {
@@ -197,7 +212,7 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
       for (int u = 0; u < 8; ++u) {
         const int pid = (u & 1) ? pid1 : pid0;
         const int c = 2 * (u >> 1);
-        if (!issue(c, c + 1, pid, pid)) return false;
+        if (!issue(true, c, c + 1, pid, pid)) return false;
       }
       return true;
     };
@@ -211,30 +226,31 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
   }
 
   if (!alive && lane == 0) {
-    // unwind: let every TMA load this warp issued land before the CTA exits
-    for (uint32_t i = 0; i < static_cast<uint32_t>(C::kSlots) && i < load_idx; ++i) {
-      const uint32_t li = load_idx - 1 - i;
-      if (static_cast<int>(li % C::kProducers) == pw)
-        drain_phase(&ct.full[li % C::kSlots], (li / C::kSlots) & 1, 1000000000ull);
-    }
+    // unwind: let every TMA load this warp issued land before the CTA exits (the latest load of
+    // each of its slots; earlier ones were consumed before the slot was refilled)
+    for (int slot = 0; slot < C::kSlots; ++slot)
+      if (mine & (1u << slot)) drain_phase(&ct.full[slot], (mine_parity >> slot) & 1u, 1000000000ull);
     if (pw == 0 && qloads > 0) drain_phase(&ct.q_full, (qloads - 1) & 1, 1000000000ull);
   }
   __syncwarp();
 }
 
-// ------------------------------------------------------------------ MMA issuer
+// ------------------------------------------------------------------ MMA issuers
+// Two threads issue MMAs: lane 0 of kMmaWarp the score products, lane 0 of kPvWarp the value
+// products.  Each commit and barrier test of an issuing thread stalls its MMA stream for a few
+// hundred cycles; two issuers hide those stalls behind each other's MMAs.  Each consumes its own
+// ring in order.  Called by lane 0 only.
 template <int N>
 __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t* qs, uint8_t* ps,
-                         uint32_t tmem, const Ctl& ctl, const int32_t* md) {
+                         uint32_t tmem, const Ctl& ctl, const int32_t* md, const bool pv_role) {
   using C = Cfg<N>;
-  if ((threadIdx.x & 31) != 0) return;
   const uint32_t idesc_qk = idesc_bf16_f32(128, N, false, false);   // K-major A (keys), K-major B (rows)
   const uint32_t idesc_pv = idesc_bf16_f32(128, N, true, true);     // MN-major A (dv), MN-major B (rows)
   const uint32_t slots_addr = smem_addr(slots);
   const uint32_t q_addr = smem_addr(qs);
   const uint32_t p_addr = smem_addr(ps);
 
-  uint32_t load_idx = 0;
+  uint32_t ridx = 0;   // loads of this issuer's ring consumed so far
   int tg = 0, qloads = 0, seg_i = 0;
   bool alive = true;
   SegIter it;
@@ -244,23 +260,26 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
   while (alive && it.next(a, s)) {
     const int tg0 = tg;
     if (s.ntiles == 0) {
-      if (seg_i > 0 && !wait_phase(&ct.o_free, (seg_i - 1) & 1, ctl)) { alive = false; break; }
+      if (pv_role && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) { alive = false; break; }
       ++seg_i;
       continue;
     }
-    if (!wait_phase(&ct.q_full, qloads & 1, ctl)) { alive = false; break; }
-    ++qloads;
-    tc_fence_after();
+    if (!pv_role) {
+      if (!wait_phase_lean(&ct.q_full, qloads & 1, ctl)) { alive = false; break; }
+      ++qloads;
+      tc_fence_after();
+    }
 
     auto do_qk = [&](int t) -> bool {
+      if (pv_role) return true;
       const int tgl = tg0 + t, sb = tgl & 1;
-      if (tgl >= 2 && !wait_phase(&ct.s_free[sb], ((tgl >> 1) - 1) & 1, ctl)) return false;
+      if (tgl >= 2 && !wait_phase_lean(&ct.s_free[sb], ((tgl >> 1) - 1) & 1, ctl)) return false;
       tc_fence_after();
       const uint32_t d_tmem = tmem + 4 * N + sb * N;
 #pragma unroll 1
       for (int c = 0; c < 9; ++c) {
-        const uint32_t slot = load_idx % C::kSlots;
-        if (!wait_phase(&ct.full[slot], (load_idx / C::kSlots) & 1, ctl)) return false;
+        const uint32_t slot = ridx % C::kSlotsQk;
+        if (!wait_phase_lean(&ct.full[slot], (ridx / C::kSlotsQk) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t base = slots_addr + slot * kSlotBytes;
 #pragma unroll
@@ -271,7 +290,7 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
           umma_bf16(d_tmem, ad, bd, idesc_qk, (c | kk) != 0 ? 1u : 0u);
         }
         umma_commit(&ct.empty[slot]);
-        ++load_idx;
+        ++ridx;
       }
       umma_commit(&ct.s_full[sb]);
       if (t == s.ntiles - 1) umma_commit(&ct.q_empty);
@@ -279,15 +298,16 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
     };
 
     auto do_pv = [&](int t) -> bool {
+      if (!pv_role) return true;
       const int tgl = tg0 + t, pb = tgl & 1;
-      if (t == 0 && seg_i > 0 && !wait_phase(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
-      if (!wait_phase(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
+      if (t == 0 && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
+      if (!wait_phase_lean(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
       tc_fence_after();
       const uint32_t pbase = p_addr + (tgl % C::kPBuf) * C::kPBytes;
 #pragma unroll 1
       for (int u = 0; u < 8; ++u) {
-        const uint32_t slot = load_idx % C::kSlots;
-        if (!wait_phase(&ct.full[slot], (load_idx / C::kSlots) & 1, ctl)) return false;
+        const uint32_t slot = C::kSlotsQk + ridx % C::kSlotsPv;
+        if (!wait_phase_lean(&ct.full[slot], (ridx / C::kSlotsPv) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t base = slots_addr + slot * kSlotBytes;
         const int q = u & 1;   // page of the tile: keys 64q .. 64q+63
@@ -300,7 +320,7 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
           umma_bf16(tmem + (u >> 1) * N, ad, bd, idesc_pv, (t > 0 || q > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&ct.empty[slot]);
-        ++load_idx;
+        ++ridx;
       }
       umma_commit(&ct.p_free[pb]);
       return true;
@@ -316,11 +336,12 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
     ++seg_i;
   }
 
-  if (!alive) {
-    // unwind: every MMA issued so far must finish before TMEM is freed
-    umma_commit(&ct.drain);
-    drain_phase(&ct.drain, 0, 1000000000ull);
-  }
+  // every MMA this thread issued has finished, and its commits have landed, before TMEM is
+  // freed and the CTA exits (on the normal path the softmax has waited for them already, but
+  // not after an abort)
+  uint64_t* drain = &ct.drain[pv_role ? 1 : 0];
+  umma_commit(drain);
+  drain_phase(drain, 0, 1000000000ull);
 }
 
 // ------------------------------------------------------------------ softmax + epilogue
@@ -581,7 +602,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     }
     mbar_init(&ct.o_free, 128);
     mbar_init(&ct.never, 1);
-    mbar_init(&ct.drain, 1);
+    mbar_init(&ct.drain[0], 1);
+    mbar_init(&ct.drain[1], 1);
     ct.abort_flag = 0;
     ct.softmax_abort = 0;
     fence_barrier_init();
@@ -605,7 +627,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   } else if (warp < C::kMmaWarp) {
     producer_role<N>(&tm_k, &tm_q, a, ct, slots, qs, ctl, rb, g, md, warp - kSoftmaxWarps);
   } else {
-    mma_role<N>(a, ct, slots, qs, ps, tmem, ctl, md);
+    if ((threadIdx.x & 31) == 0) mma_role<N>(a, ct, slots, qs, ps, tmem, ctl, md, warp == C::kPvWarp);
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -30,19 +30,23 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
+// The waits and arrives use the instructions' default memory semantics
+// (acquire and release at CTA scope). Spelling the same semantics out as
+// `.acquire.cta` made each completed-phase test cost about 900 cycles behind
+// in-flight MMAs instead of about 150, so the qualifiers are left implicit.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(done) : "r"(smem_addr(bar)), "r"(parity) : "memory");
   return done != 0;
@@ -89,6 +93,17 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, const
   }
 }
 
+// The same wait for MMA-issuing threads: the first test inline, the polling
+// loop out of line.  With the loop inlined next to tcgen05.mma, every MMA of
+// the issuing loop costs several times its pipe time, even when the loop is
+// never entered.
+static __device__ __noinline__ bool wait_phase_slow(uint64_t* bar, uint32_t parity, const Ctl& c) {
+  return wait_phase(bar, parity, c);
+}
+__device__ __forceinline__ bool wait_phase_lean(uint64_t* bar, uint32_t parity, const Ctl& c) {
+  return mbar_test(bar, parity) || wait_phase_slow(bar, parity, c);
+}
+
 // Bounded wait used only while unwinding: ignores the abort flag.
 __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
@@ -98,16 +113,12 @@ __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity, uint
   return true;
 }
 
-// Same wait, with cluster-scope acquire: for barriers that threads of the
-// peer CTA arrive on remotely.
+// Wait on a barrier that threads of the peer CTA arrive on remotely. The
+// data those arrivals publish is read by the tensor cores of the CTA that
+// wrote it (its half of a paired MMA operand) and was fenced into the async
+// proxy before the arrive, so the default-scope test suffices.
 __device__ __forceinline__ bool mbar_test_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-  return done != 0;
+  return mbar_test(bar, parity);
 }
 
 __device__ __forceinline__ bool wait_phase_cluster(uint64_t* bar, uint32_t parity, const Ctl& c) {

@@ -147,6 +147,36 @@ def test_full_size_configs_sampled(index):
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
 
 
+@pytest.mark.parametrize("rows", [16, 32, 64, 128])
+def test_repeated_launches_are_bit_identical(rows):
+    """Hundreds of back-to-back launches on the varlen lengths of the memory-bound
+    workload, with short wait limits: every launch finishes without a timeout and
+    reproduces the first bit for bit.  Pipeline races between the roles of a CTA
+    (a barrier phase taken for the wrong load) show up here as timeouts or as
+    launches that differ."""
+    w = inputs.build(f"repeat{rows}", inputs.config_seqlens(3), s_q=1, h_q=rows, seed=90 + rows)
+    q, k, bt, sl = to_gpu(w)
+    md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(binding.workspace_bytes(w.batch, w.rows_per_kv, w.h_kv, md.shape[0]),
+                     dtype=torch.uint8, device="cuda")
+    out0, lse0 = binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, workspace=ws,
+                                      status=status, timeout_ns=200_000_000)
+    out0, lse0 = out0.clone(), lse0.clone()
+    out, lse = torch.empty_like(out0), torch.empty_like(lse0)
+    bad = torch.zeros((), dtype=torch.int64, device="cuda")
+    for _ in range(300):
+        binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, workspace=ws, out=out, lse=lse,
+                             status=status, timeout_ns=200_000_000)
+        bad += (out.view(torch.int16) != out0.view(torch.int16)).any() | (lse.view(torch.int32) != lse0.view(torch.int32)).any()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, binding.status_string(int(status.item()))
+    assert int(bad.item()) == 0
+    sample = [0, w.batch // 2, w.batch - 1]
+    o_ref, l_ref = oracle(w, batches=sample)
+    compare(w, out0, lse0, o_ref, l_ref, batches=sample, what=f"repeat rows={rows}")
+
+
 # ---------------------------------------------------------------- failure paths
 
 def test_bounded_wait_reports_timeout_and_context_survives():
