@@ -47,7 +47,7 @@ constexpr int kKSlots = 3;             // score ring: three chunks of this CTA's
 constexpr int kKSlotBytes = 3 * kBox;
 constexpr int kVSlots = 2;             // value ring: [dv half][2 chunks] of one page per slot
 constexpr int kVSlotBytes = 4 * kBox;
-constexpr int kThreads = 224;          // warps 0-3 softmax, 4 score loads, 5 value loads, 6 MMA
+constexpr int kThreads = 256;          // warps 0-3 softmax, 4 score loads, 5 value loads, 6-7 MMA issuers
 constexpr int kQBytes = 9 * kBox;      // 64 rows x 576: [chunk][row][64 cols]
 constexpr int kPBytes = 2 * kBox;      // P: [key half][64 rows][64 keys] bf16 (one buffer)
 constexpr int kOffP = kQBytes;
@@ -68,7 +68,7 @@ struct Ctrl {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
-  uint64_t o_free, never, drain;
+  uint64_t o_free, never, drain[2];
   uint32_t tmem_base;
   int abort_flag;
   int softmax_abort;
@@ -216,9 +216,12 @@ __device__ void value_loads(const PairMaps& maps, const DecodeArgs& a, Ctrl& ct,
   __syncwarp();
 }
 
-// ------------------------------------------------------------------ MMA (leader CTA, one thread)
+// ------------------------------------------------------------------ MMA (leader CTA, two threads)
+// Lane 0 of warp 6 issues the score products (it consumes the score ring), lane 0 of warp 7 the
+// value products (the value ring): the commit and barrier stalls of one issuer are hidden behind
+// the other's MMAs.
 __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* ps, uint8_t* ks, uint8_t* vs,
-                          uint32_t tmem, const Ctl& ctl, const int32_t* md) {
+                          uint32_t tmem, const Ctl& ctl, const int32_t* md, const bool pv_role) {
   const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);   // A = Q (K-major), B = K (K-major)
   const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);    // A = P (K-major), B = V (MN-major)
   const uint32_t q_addr = smem_addr(qs), p_addr = smem_addr(ps), k_addr = smem_addr(ks), v_addr = smem_addr(vs);
@@ -230,23 +233,26 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
   while (it.next(a, s)) {
     const int tg0 = tg;
     if (s.ntiles == 0) {
-      if (seg_i > 0 && !wait_phase_cluster(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
+      if (pv_role && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
       ++seg_i;
       continue;
     }
-    if (!wait_phase(&ct.q_full, qloads & 1, ctl)) return false;
-    ++qloads;
-    tc_fence_after();
+    if (!pv_role) {
+      if (!wait_phase_lean(&ct.q_full, qloads & 1, ctl)) return false;
+      ++qloads;
+      tc_fence_after();
+    }
 
     auto do_qk = [&](int t) -> bool {
+      if (pv_role) return true;
       const int tgl = tg0 + t, sb = tgl & 1;
-      if (tgl >= 2 && !wait_phase_cluster(&ct.s_free[sb], ((tgl >> 1) - 1) & 1, ctl)) return false;
+      if (tgl >= 2 && !wait_phase_lean(&ct.s_free[sb], ((tgl >> 1) - 1) & 1, ctl)) return false;
       tc_fence_after();
       const uint32_t d_tmem = tmem + kColS + 64 * sb;
 #pragma unroll 1
       for (int j = 0; j < 3; ++j) {
         const uint32_t slot = kidx % kKSlots;
-        if (!wait_phase(&ct.k_full[slot], (kidx / kKSlots) & 1, ctl)) return false;
+        if (!wait_phase_lean(&ct.k_full[slot], (kidx / kKSlots) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 3; ++cc) {
@@ -266,14 +272,15 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
     };
 
     auto do_pv = [&](int t) -> bool {
+      if (!pv_role) return true;
       const int tgl = tg0 + t, pb = tgl & 1;
-      if (t == 0 && seg_i > 0 && !wait_phase_cluster(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
-      if (!wait_phase_cluster(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
+      if (t == 0 && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
+      if (!wait_phase_lean(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
       tc_fence_after();
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {       // page q of the tile
         const uint32_t slot = vidx % kVSlots;
-        if (!wait_phase(&ct.v_full[slot], (vidx / kVSlots) & 1, ctl)) return false;
+        if (!wait_phase_lean(&ct.v_full[slot], (vidx / kVSlots) & 1, ctl)) return false;
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {     // dv half
@@ -534,7 +541,8 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
     }
     mbar_init(&ct.o_free, 8);
     mbar_init(&ct.never, 1);
-    mbar_init(&ct.drain, 1);
+    mbar_init(&ct.drain[0], 1);
+    mbar_init(&ct.drain[1], 1);
     ct.abort_flag = 0;
     ct.softmax_abort = 0;
     fence_barrier_init();
@@ -563,19 +571,22 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
   const uint32_t L_p_full0 = mapa_shared(smem_addr(&ct.p_full[0]), 0);
   const uint32_t L_o_free = mapa_shared(smem_addr(&ct.o_free), 0);
 
-  bool clean = true;
   if (warp < 4) {
     softmax_rows(a, ct, ps, tmem, ctl, rank, rb, g, md, L_s_free0, L_p_full0, L_o_free);
   } else if (warp == 4) {
     score_loads(maps, a, ct, qs, ks, ctl, rank, rb, g, md, L_q_full, L_k_full0);
   } else if (warp == 5) {
     value_loads(maps, a, ct, vs, ctl, rank, g, md, L_v_full0);
-  } else if (rank == 0 && (threadIdx.x & 31) == 0) {
-    clean = mma_issue(a, ct, qs, ps, ks, vs, tmem, ctl, md);
-    if (!clean) {
-      umma_commit_pair(&ct.drain);      // every MMA issued so far has finished before TMEM is freed
-      drain_phase(&ct.drain, 0, 1000000000ull);
+  } else {
+    if (rank == 0 && (threadIdx.x & 31) == 0) {
+      const bool pv_role = warp == 7;
+      (void)mma_issue(a, ct, qs, ps, ks, vs, tmem, ctl, md, pv_role);
+      // every MMA this thread issued has finished, and its commits have landed, before TMEM is
+      // freed and the pair exits (the softmax has waited for them unless the pair is aborting)
+      umma_commit_pair_leader(&ct.drain[pv_role ? 1 : 0]);
+      drain_phase(&ct.drain[pv_role ? 1 : 0], 0, 1000000000ull);
     }
+    __syncwarp();
   }
   __syncthreads();
   if (ct.abort_flag) settle_ns(200000);   // let loads already issued land before the pair exits

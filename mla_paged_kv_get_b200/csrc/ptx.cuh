@@ -335,6 +335,15 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
 
 // Arrive once on the barrier at the same offset in both CTAs of the pair when
 // every pair MMA issued so far by this thread has completed.
+// Completion of this thread's paired MMAs, signalled on the leader CTA's barrier only.
+__device__ __forceinline__ void umma_commit_pair_leader(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 1;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}\n"
+      ::"r"(smem_addr(bar)) : "memory");
+}
+
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .b16 m;\n\t"
