@@ -177,6 +177,45 @@ def test_repeated_launches_are_bit_identical(rows):
     compare(w, out0, lse0, o_ref, l_ref, batches=sample, what=f"repeat rows={rows}")
 
 
+def test_step_replays_from_a_cuda_graph():
+    """Metadata, decode and combine are stream-ordered with no host synchronisation,
+    so one decode step captures into a CUDA graph; replays on new cache lengths and
+    contents give what eager calls give, bit for bit."""
+    w = inputs.config(3)
+    q, k, bt, sl = to_gpu(w)
+    G = binding.num_parts(w.rows_per_kv, w.h_kv)
+    ws = torch.empty(binding.workspace_bytes(w.batch, w.rows_per_kv, w.h_kv, G), dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.batch, w.s_q, w.h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv)
+        binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, workspace=ws, out=out, lse=lse,
+                             status=status)
+
+    step()                                   # first call sets the kernels' shared-memory attributes
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for trial in range(3):
+        # new lengths (same page table capacity) and new cache values, written in place
+        g = torch.Generator().manual_seed(500 + trial)
+        new_len = torch.randint(1, 64 * bt.shape[1] + 1, (w.batch,), generator=g, dtype=torch.int32)
+        sl.copy_(new_len.cuda())
+        k.copy_((torch.randn(k.shape, generator=g) * 0.5).to(torch.bfloat16).cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        got_out, got_lse = out.clone(), lse.clone()
+        step()
+        torch.cuda.synchronize()
+        assert torch.equal(got_out.view(torch.int16), out.view(torch.int16))
+        assert torch.equal(got_lse.view(torch.int32), lse.view(torch.int32))
+    del graph
+
+
 # ---------------------------------------------------------------- failure paths
 
 def test_bounded_wait_reports_timeout_and_context_survives():
