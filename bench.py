@@ -212,6 +212,47 @@ def cpu_oracle_timing(w, budget_s: float = 15.0):
             "hbm_equiv_gbs": done_bytes / dt / 1e9, "seconds": dt}
 
 
+def torch_native_timing(w, q, k, bt, sl, flops: int, reps: int = 10):
+    """The same decode in plain PyTorch on the GPU, timed next to the kernels.
+
+    Dense page gather through the block table, S = scale * Q.K^T (bf16 matmul), the
+    length (and causal) mask, softmax in fp32, O = P.V with V the first 512 columns,
+    and the logsumexp.  A same-box comparison on the same algorithmic work, not a
+    path the library ever takes.
+    """
+    B, s_q, h_q, h_kv = w.batch, w.s_q, w.h_q, w.h_kv
+    hg = h_q // h_kv
+    T = bt.shape[1] * 64
+    j = torch.arange(T, device=q.device)
+    srow = torch.arange(s_q, device=q.device).repeat_interleave(hg)                # row -> query token
+    lim = sl.long()[:, None] - ((s_q - 1 - srow)[None, :] if w.causal else 0)      # [B, rows]
+    valid = (j[None, None, :] < lim[:, :, None])[:, None]                          # [B, 1, rows, T]
+
+    def run():
+        kd = k[bt.long()].reshape(B, T, h_kv, 576).permute(0, 2, 1, 3)             # [B, h_kv, T, 576]
+        qg = q.reshape(B, s_q, h_kv, hg, 576).permute(0, 2, 1, 3, 4).reshape(B, h_kv, s_q * hg, 576)
+        s = torch.matmul(qg, kd.transpose(-1, -2)).float() * w.scale
+        s = s.masked_fill(~valid, float("-inf"))
+        lse = torch.logsumexp(s, dim=-1)
+        p = torch.softmax(s, dim=-1).to(q.dtype)
+        o = torch.matmul(p, kd[..., :512])
+        return o, lse
+
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "reps": reps,
+            "what": "PyTorch on this GPU: dense page gather, bf16 matmul Q.K^T, masked fp32 softmax and "
+                    "logsumexp, bf16 matmul P.V (a comparison; the library never takes this path)"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -247,6 +288,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-torch-baseline", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
@@ -408,6 +450,8 @@ def main(argv=None):
         "gpu_launches": 3 * args.steps,
         "clocks": sampler.summary(),
     }
+    if rank == 0 and world == 1 and not args.no_torch_baseline:
+        line["torch_baseline"] = torch_native_timing(w, q, k, bt, sl, flops)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_timing(w)
     if rank == 0:

@@ -42,6 +42,10 @@ extern "C" {
 #define MLA_ERR_TIMEOUT      -5   /* device-side bounded wait gave up (status_d) */
 #define MLA_ERR_BAD_INPUT    -6   /* device-side input check failed (status_d)   */
 
+/* Element type of q, k_cache and out (kind::f16 MMAs accumulate in fp32 for both). */
+#define MLA_DTYPE_BF16  0
+#define MLA_DTYPE_FP16  1
+
 #define MLA_HEAD_DIM   576
 #define MLA_VALUE_DIM  512
 #define MLA_PAGE_SIZE  64
@@ -156,6 +160,28 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages,
  */
 int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch,
                 int s_q, int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream);
+
+/*
+ * mla_decode_paged_ex and mla_combine for either element type.  The pages list
+ * FP16 next to BF16 among the kernel's data types (cnblogs §2 关键特性); the
+ * release notes on every page name BF16, which the calls above use.
+ *   dtype   MLA_DTYPE_BF16 or MLA_DTYPE_FP16: the type of q_d, k_cache_d and
+ *           out_d (2 bytes per element either way; same layouts and alignment
+ *           rules).  P is rounded to the same type before the value product.
+ * Other arguments and results exactly as mla_decode_paged_ex / mla_combine;
+ * MLA_ERR_INVALID_ARG for any other dtype.
+ */
+int mla_decode_paged_typed(int dtype, const void* q_d, const void* k_cache_d, int num_pages,
+                           const int32_t* block_table_d, int max_pages_per_seq,
+                           const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
+                           int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d,
+                           int num_parts, int causal, float softmax_scale,
+                           void* workspace_d, size_t workspace_bytes,
+                           void* out_d, float* lse_d, int32_t* status_d,
+                           int debug_flags, unsigned long long timeout_ns, void* stream);
+int mla_combine_typed(int dtype, const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes,
+                      int batch, int s_q, int h_q, int h_kv, int num_parts, void* out_d, float* lse_d,
+                      void* stream);
 
 /*
  * Allocation-free variant of mla_decode_paged.  The pages describe no such

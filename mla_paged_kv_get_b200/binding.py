@@ -74,6 +74,10 @@ def load_library() -> ctypes.CDLL:
     lib.mla_decode_paged_ex.argtypes = dec + [ci, ctypes.c_ulonglong, vp]
     lib.mla_decode_paged_ex.restype = ci
     lib.mla_combine.argtypes = [i32p, vp, csz, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.mla_decode_paged_typed.argtypes = [ci] + dec + [ci, ctypes.c_ulonglong, vp]
+    lib.mla_decode_paged_typed.restype = ci
+    lib.mla_combine_typed.argtypes = [ci, i32p, vp, csz, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.mla_combine_typed.restype = ci
     lib.mla_combine.restype = ci
     _lib = lib
     return lib
@@ -95,6 +99,10 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+# element types of q / k_cache / out and their codes in the C ABI (MLA_DTYPE_*)
+DTYPES = {torch.bfloat16: 0, torch.float16: 1}
 
 
 def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
@@ -146,10 +154,14 @@ def decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tens
                  softmax_scale: float | None = None, workspace: torch.Tensor | None = None,
                  out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                  status: torch.Tensor | None = None, debug_flags: int = 0, timeout_ns: int = 0, stream=None):
-    """MLA decode over the paged cache; returns ``(out [B,s_q,h_q,dv] bf16, lse [B,s_q,h_q] fp32)``."""
+    """MLA decode over the paged cache; returns ``(out [B,s_q,h_q,dv], lse [B,s_q,h_q] fp32)``.
+
+    q and k_cache are both bf16 or both fp16; out has their type."""
     lib = load_library()
-    _need(q, "q", torch.bfloat16)
-    _need(k_cache, "k_cache", torch.bfloat16)
+    if q.dtype not in DTYPES:
+        raise ValueError(f"q must be bf16 or fp16, got {q.dtype}")
+    _need(q, "q", q.dtype)
+    _need(k_cache, "k_cache", q.dtype)
     _need(block_table, "block_table", torch.int32)
     _need(cache_seqlens, "cache_seqlens", torch.int32)
     _need(tile_md, "tile_md", torch.int32)
@@ -167,11 +179,12 @@ def decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tens
     if workspace is None:
         workspace = torch.empty((workspace_bytes(B, R, h_kv, G, dv),), dtype=torch.uint8, device=q.device)
     if out is None:
-        out = torch.empty((B, s_q, h_q, dv), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, s_q, h_q, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype)
     if lse is None:
         lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=q.device)
-    code = lib.mla_decode_paged_ex(
-        _ptr(q), _ptr(k_cache), num_pages, _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
+    code = lib.mla_decode_paged_typed(
+        DTYPES[q.dtype], _ptr(q), _ptr(k_cache), num_pages, _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
         B, s_q, h_q, h_kv, d, dv, _ptr(tile_md), _ptr(num_splits), G, int(bool(causal)), float(softmax_scale),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse), _ptr(status),
         int(debug_flags), int(timeout_ns), _stream_handle(stream))

@@ -128,12 +128,15 @@ size_t mla_workspace_bytes(int batch, int rows_per_kv, int h_kv, int dv, int num
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
-int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, const int32_t* block_table_d,
-                        int max_pages_per_seq, const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
-                        int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d, int num_parts,
-                        int causal, float softmax_scale, void* workspace_d, size_t workspace_bytes, void* out_d,
-                        float* lse_d, int32_t* status_d, int debug_flags, unsigned long long timeout_ns,
-                        void* stream) {
+int mla_decode_paged_typed(int dtype, const void* q_d, const void* k_cache_d, int num_pages,
+                           const int32_t* block_table_d, int max_pages_per_seq, const int32_t* cache_seqlens_d,
+                           int batch, int s_q, int h_q, int h_kv, int d, int dv, const int32_t* tile_md_d,
+                           const int32_t* num_splits_d, int num_parts, int causal, float softmax_scale,
+                           void* workspace_d, size_t workspace_bytes, void* out_d, float* lse_d, int32_t* status_d,
+                           int debug_flags, unsigned long long timeout_ns, void* stream) {
+  if (dtype != MLA_DTYPE_BF16 && dtype != MLA_DTYPE_FP16) return MLA_ERR_INVALID_ARG;
+  const CUtensorMapDataType tmap_type =
+      dtype == MLA_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (q_d == nullptr || k_cache_d == nullptr || block_table_d == nullptr || cache_seqlens_d == nullptr ||
       tile_md_d == nullptr || num_splits_d == nullptr || out_d == nullptr || lse_d == nullptr)
     return MLA_ERR_INVALID_ARG;
@@ -172,7 +175,7 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
     const cuuint64_t strides[3] = {token_bytes, 128, MLA_HEAD_DIM * 2ull};
     const cuuint32_t box[4] = {64, 64, static_cast<cuuint32_t>(chunks), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k_cache_d), dims, strides, box, estr,
+    return encode(m, tmap_type, 4, const_cast<void*>(k_cache_d), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
@@ -187,7 +190,7 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
                                    static_cast<cuuint64_t>(h_q) * MLA_HEAD_DIM * 2ull, 128};
     const cuuint32_t box[5] = {64, static_cast<cuuint32_t>(bh), 1, static_cast<cuuint32_t>(bs), 9};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q_d), dims, strides, box, estr,
+    return encode(m, tmap_type, 5, const_cast<void*>(q_d), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
@@ -198,7 +201,7 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
   a.seqlens = cache_seqlens_d;
   a.tile_md = tile_md_d;
   a.num_splits = num_splits_d;
-  a.out = static_cast<__nv_bfloat16*>(out_d);
+  a.out = out_d;
   a.lse = lse_d;
   const size_t max_pieces = static_cast<size_t>(batch) + num_parts;
   a.o_part = static_cast<float*>(workspace_d);
@@ -234,28 +237,30 @@ int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, c
       const cuuint32_t box[5] = {64, 64, 2, 2, 1};
       const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
       void* base = static_cast<char*>(const_cast<void*>(k_cache_d)) + 256 * rank;
-      if (encode(&maps.v[rank], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
+      if (encode(&maps.v[rank], tmap_type, 5, base, dims, strides, box, estr,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return MLA_ERR_CUDA;
     }
     if (!q_map(&maps.q, 64)) return MLA_ERR_CUDA;
-    le = mla::launch_decode_pair(maps, a, row_blocks, s);
+    le = mla::launch_decode_pair(dtype, maps, a, row_blocks, s);
   } else {
     CUtensorMap tm_k, tm_q;
     if (!page_map(&tm_k, 1) || !q_map(&tm_q, n)) return MLA_ERR_CUDA;
-    le = mla::launch_decode(n, tm_k, tm_q, a, row_blocks, s);
+    le = mla::launch_decode(n, dtype, tm_k, tm_q, a, row_blocks, s);
   }
   if (le != cudaSuccess) return MLA_ERR_CUDA;
   if (debug_flags & 2) return MLA_OK;
-  if (mla::launch_combine(num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=
+  if (mla::launch_combine(dtype, num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
 }
 
-int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch, int s_q,
-                int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream) {
+int mla_combine_typed(int dtype, const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes,
+                      int batch, int s_q, int h_q, int h_kv, int num_parts, void* out_d, float* lse_d,
+                      void* stream) {
+  if (dtype != MLA_DTYPE_BF16 && dtype != MLA_DTYPE_FP16) return MLA_ERR_INVALID_ARG;
   if (num_splits_d == nullptr || workspace_d == nullptr || out_d == nullptr || lse_d == nullptr)
     return MLA_ERR_INVALID_ARG;
   if (batch < 1 || batch > 65535 || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || num_parts < 1)
@@ -266,10 +271,28 @@ int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t wor
   const size_t max_pieces = static_cast<size_t>(batch) + num_parts;
   const float* o_part = static_cast<const float*>(workspace_d);
   const float* lse_part = o_part + max_pieces * h_kv * R * MLA_VALUE_DIM;
-  if (mla::launch_combine(num_splits_d, o_part, lse_part, static_cast<__nv_bfloat16*>(out_d), lse_d, batch, s_q,
-                          h_q, h_kv, R, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (mla::launch_combine(dtype, num_splits_d, o_part, lse_part, out_d, lse_d, batch, s_q, h_q, h_kv, R,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
+}
+
+int mla_combine(const int32_t* num_splits_d, const void* workspace_d, size_t workspace_bytes, int batch, int s_q,
+                int h_q, int h_kv, int num_parts, void* out_d, float* lse_d, void* stream) {
+  return mla_combine_typed(MLA_DTYPE_BF16, num_splits_d, workspace_d, workspace_bytes, batch, s_q, h_q, h_kv,
+                           num_parts, out_d, lse_d, stream);
+}
+
+int mla_decode_paged_ex(const void* q_d, const void* k_cache_d, int num_pages, const int32_t* block_table_d,
+                        int max_pages_per_seq, const int32_t* cache_seqlens_d, int batch, int s_q, int h_q, int h_kv,
+                        int d, int dv, const int32_t* tile_md_d, const int32_t* num_splits_d, int num_parts,
+                        int causal, float softmax_scale, void* workspace_d, size_t workspace_bytes, void* out_d,
+                        float* lse_d, int32_t* status_d, int debug_flags, unsigned long long timeout_ns,
+                        void* stream) {
+  return mla_decode_paged_typed(MLA_DTYPE_BF16, q_d, k_cache_d, num_pages, block_table_d, max_pages_per_seq,
+                                cache_seqlens_d, batch, s_q, h_q, h_kv, d, dv, tile_md_d, num_splits_d, num_parts,
+                                causal, softmax_scale, workspace_d, workspace_bytes, out_d, lse_d, status_d,
+                                debug_flags, timeout_ns, stream);
 }
 
 int mla_decode_paged(const void* q_d, const void* k_cache_d, int num_pages, const int32_t* block_table_d,

@@ -10,8 +10,9 @@
 // skipped here.
 //
 // One warp per query row: each lane owns 16 of the 512 values, reads them with
-// 16-byte loads per piece and writes 16 bf16 (two 16-byte stores), so a warp
+// 16-byte loads per piece and writes 16 output values (two 16-byte stores), so a warp
 // moves whole 2 KB partial rows and a 1 KB output row.
+#include "ptx.cuh"
 #include "decode.cuh"
 
 namespace mla {
@@ -20,9 +21,10 @@ namespace {
 
 constexpr int kRowsPerBlock = 4;
 
+template <int T>
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
 mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restrict__ o_part,
-                   const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ out,
+                   const float* __restrict__ lse_part, uint16_t* __restrict__ out,
                    float* __restrict__ lse, int batch, int s_q, int h_q, int h_kv, int R) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kRowsPerBlock + warp;
@@ -71,8 +73,7 @@ mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restri
   uint32_t packed[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    packed[i] = *reinterpret_cast<uint32_t*>(&v);
+    packed[i] = pack2<T>(acc[2 * i], acc[2 * i + 1]);
   }
   uint4* dst = reinterpret_cast<uint4*>(out + out_row * 512) + lane * 2;
   dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
@@ -82,12 +83,17 @@ mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restri
 
 }  // namespace
 
-cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
-                           __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
+cudaError_t launch_combine(int dtype, const int32_t* num_splits, const float* o_part, const float* lse_part,
+                           void* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
                            cudaStream_t stream) {
   const dim3 grid((R + kRowsPerBlock - 1) / kRowsPerBlock, h_kv, batch);
-  mla_combine_kernel<<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, out, lse, batch,
-                                                              s_q, h_q, h_kv, R);
+  uint16_t* o = static_cast<uint16_t*>(out);
+  if (dtype == kFP16)
+    mla_combine_kernel<kFP16><<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, o, lse, batch,
+                                                                     s_q, h_q, h_kv, R);
+  else
+    mla_combine_kernel<kBF16><<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, o, lse, batch,
+                                                                     s_q, h_q, h_kv, R);
   return cudaGetLastError();
 }
 

@@ -240,12 +240,12 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
 // products.  Each commit and barrier test of an issuing thread stalls its MMA stream for a few
 // hundred cycles; two issuers hide those stalls behind each other's MMAs.  Each consumes its own
 // ring in order.  Called by lane 0 only.
-template <int N>
+template <int N, int T>
 __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t* qs, uint8_t* ps,
                          uint32_t tmem, const Ctl& ctl, const int32_t* md, const bool pv_role) {
   using C = Cfg<N>;
-  const uint32_t idesc_qk = idesc_bf16_f32(128, N, false, false);   // K-major A (keys), K-major B (rows)
-  const uint32_t idesc_pv = idesc_bf16_f32(128, N, true, true);     // MN-major A (dv), MN-major B (rows)
+  const uint32_t idesc_qk = idesc_f32<T>(128, N, false, false);   // K-major A (keys), K-major B (rows)
+  const uint32_t idesc_pv = idesc_f32<T>(128, N, true, true);     // MN-major A (dv), MN-major B (rows)
   const uint32_t slots_addr = smem_addr(slots);
   const uint32_t q_addr = smem_addr(qs);
   const uint32_t p_addr = smem_addr(ps);
@@ -345,7 +345,7 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
 }
 
 // ------------------------------------------------------------------ softmax + epilogue
-template <int N>
+template <int N, int T>
 __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_t tmem, const Ctl& ctl,
                              int rb, int g, const int32_t* md) {
   using C = Cfg<N>;
@@ -475,9 +475,9 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
           const int c = 8 * c8 + 2 * i;
           const float p0 = x[c] == -INFINITY ? 0.f : ex2(x[c] - ct.m_run[c]);
           const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2(x[c + 1] - ct.m_run[c + 1]);
-          w[i] = pack_bf16(p0, p1);
-          lsum[c] += __uint_as_float(w[i] << 16);
-          lsum[c + 1] += __uint_as_float(w[i] & 0xffff0000u);
+          w[i] = pack2<T>(p0, p1);
+          lsum[c] += unpack_lo<T>(w[i]);
+          lsum[c + 1] += unpack_hi<T>(w[i]);
         }
         const uint32_t off = static_cast<uint32_t>(tid * 2 * N + c8 * 16);
         const uint32_t phys = off ^ (((off >> 7) & C::kPSwizzleMask) << 4);
@@ -514,7 +514,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
     const bool final_out = npieces == 1;
     const bool can_write = final_out || s.piece < a.max_pieces;
     if (!can_write && tid == 0) record_status(a.status, MLA_ERR_BAD_INPUT);
-    __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(ps);
+    uint16_t* stage_h = reinterpret_cast<uint16_t*>(ps);
 
 #pragma unroll 1
     for (int d = 0; d < 4; ++d) {
@@ -535,7 +535,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
       if (final_out) {
         // stage [row][128 dv] bf16 (one P buffer) so each output row slice leaves as 16-byte vectors
 #pragma unroll
-        for (int c = 0; c < N; ++c) stage_h[c * 128 + tid] = __float2bfloat16_rn(v[c] * ct.inv_l[c]);
+        for (int c = 0; c < N; ++c) stage_h[c * 128 + tid] = to_bits<T>(v[c] * ct.inv_l[c]);
         named_sync(kSoftmaxBar, 128);
         if (can_write) {
           for (int i = tid; i < rows_here * 16; i += 128) {
@@ -543,7 +543,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
             const int r = rb * N + c;
             const int srow = r / hg, h = g * hg + r % hg;
             const uint4 val = reinterpret_cast<const uint4*>(ps)[c * 16 + vv];
-            __nv_bfloat16* dst = a.out + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + h) * 512 + d * 128;
+            uint16_t* dst = static_cast<uint16_t*>(a.out) + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + h) * 512 + d * 128;
             reinterpret_cast<uint4*>(dst)[vv] = val;
           }
         }
@@ -571,7 +571,7 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
   }
 }
 
-template <int N>
+template <int N, int T>
 __global__ void __launch_bounds__(Cfg<N>::kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const DecodeArgs a) {
@@ -623,11 +623,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const Ctl ctl{&ct.abort_flag, a.status, a.timeout_ns};
 
   if (warp < kSoftmaxWarps) {
-    softmax_role<N>(a, ct, ps, tmem, ctl, rb, g, md);
+    softmax_role<N, T>(a, ct, ps, tmem, ctl, rb, g, md);
   } else if (warp < C::kMmaWarp) {
     producer_role<N>(&tm_k, &tm_q, a, ct, slots, qs, ctl, rb, g, md, warp - kSoftmaxWarps);
   } else {
-    if ((threadIdx.x & 31) == 0) mma_role<N>(a, ct, slots, qs, ps, tmem, ctl, md, warp == C::kPvWarp);
+    if ((threadIdx.x & 31) == 0) mma_role<N, T>(a, ct, slots, qs, ps, tmem, ctl, md, warp == C::kPvWarp);
     __syncwarp();
   }
 
@@ -650,31 +650,38 @@ int decode_smem_bytes(int n) {
   }
 }
 
-template <int N>
+template <int N, int T>
 static cudaError_t launch_n(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, dim3 grid,
                             cudaStream_t stream) {
   static int configured_device = -1;   // attribute is per device; re-set if the device changes
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<N, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<N>::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  mla_decode_kernel<N><<<grid, Cfg<N>::kThreads, Cfg<N>::kSmemBytes, stream>>>(tm_k, tm_q, a);
+  mla_decode_kernel<N, T><<<grid, Cfg<N>::kThreads, Cfg<N>::kSmemBytes, stream>>>(tm_k, tm_q, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(int n, const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a,
-                          int row_blocks, cudaStream_t stream) {
-  const dim3 grid(row_blocks, a.h_kv, a.num_parts);
+template <int T>
+static cudaError_t launch_t(int n, const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, dim3 grid,
+                            cudaStream_t stream) {
   switch (n) {
-    case 16: return launch_n<16>(tm_k, tm_q, a, grid, stream);
-    case 32: return launch_n<32>(tm_k, tm_q, a, grid, stream);
-    case 64: return launch_n<64>(tm_k, tm_q, a, grid, stream);
+    case 16: return launch_n<16, T>(tm_k, tm_q, a, grid, stream);
+    case 32: return launch_n<32, T>(tm_k, tm_q, a, grid, stream);
+    case 64: return launch_n<64, T>(tm_k, tm_q, a, grid, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_decode(int n, int dtype, const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a,
+                          int row_blocks, cudaStream_t stream) {
+  const dim3 grid(row_blocks, a.h_kv, a.num_parts);
+  if (dtype == kFP16) return launch_t<kFP16>(n, tm_k, tm_q, a, grid, stream);
+  return launch_t<kBF16>(n, tm_k, tm_q, a, grid, stream);
 }
 
 }  // namespace mla

@@ -15,7 +15,7 @@ struct DecodeArgs {
   const int32_t* seqlens;       // [batch]
   const int32_t* tile_md;       // [num_parts, 8]
   const int32_t* num_splits;    // [batch + 1]
-  __nv_bfloat16* out;           // [batch, s_q, h_q, 512]
+  void* out;                    // [batch, s_q, h_q, 512] bf16 or fp16
   float* lse;                   // [batch, s_q, h_q]
   float* o_part;                // [max_pieces, h_kv, R, 512]
   float* lse_part;              // [max_pieces, h_kv, R]
@@ -28,7 +28,8 @@ struct DecodeArgs {
 };
 
 int decode_smem_bytes(int rows_per_block);
-cudaError_t launch_decode(int rows_per_block, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+// dtype: MLA_DTYPE_BF16 or MLA_DTYPE_FP16 (q, cache and out)
+cudaError_t launch_decode(int rows_per_block, int dtype, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                           const DecodeArgs& a, int row_blocks, cudaStream_t stream);
 
 // Tensor maps of the pair kernel: the score product's page chunks (24 KB boxes),
@@ -40,10 +41,11 @@ struct PairMaps {
 };
 
 int decode_pair_smem_bytes();
-cudaError_t launch_decode_pair(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream);
+cudaError_t launch_decode_pair(int dtype, const PairMaps& maps, const DecodeArgs& a, int row_blocks,
+                               cudaStream_t stream);
 
-cudaError_t launch_combine(const int32_t* num_splits, const float* o_part, const float* lse_part,
-                           __nv_bfloat16* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
+cudaError_t launch_combine(int dtype, const int32_t* num_splits, const float* o_part, const float* lse_part,
+                           void* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
                            cudaStream_t stream);
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,

@@ -220,10 +220,11 @@ __device__ void value_loads(const PairMaps& maps, const DecodeArgs& a, Ctrl& ct,
 // Lane 0 of warp 6 issues the score products (it consumes the score ring), lane 0 of warp 7 the
 // value products (the value ring): the commit and barrier stalls of one issuer are hidden behind
 // the other's MMAs.
+template <int T>
 __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* ps, uint8_t* ks, uint8_t* vs,
                           uint32_t tmem, const Ctl& ctl, const int32_t* md, const bool pv_role) {
-  const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);   // A = Q (K-major), B = K (K-major)
-  const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);    // A = P (K-major), B = V (MN-major)
+  const uint32_t idesc_qk = idesc_f32<T>(128, 128, false, false);   // A = Q (K-major), B = K (K-major)
+  const uint32_t idesc_pv = idesc_f32<T>(128, 256, false, true);    // A = P (K-major), B = V (MN-major)
   const uint32_t q_addr = smem_addr(qs), p_addr = smem_addr(ps), k_addr = smem_addr(ks), v_addr = smem_addr(vs);
   uint32_t kidx = 0, vidx = 0;
   int tg = 0, qloads = 0, seg_i = 0;
@@ -313,6 +314,7 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
 }
 
 // ------------------------------------------------------------------ softmax + epilogue (warps 0-3)
+template <int T>
 __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_t tmem, const Ctl& ctl,
                              uint32_t rank, int rb, int g, const int32_t* md, uint32_t leader_s_free0,
                              uint32_t leader_p_full0, uint32_t leader_o_free) {
@@ -430,8 +432,8 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = 8 * c8 + 2 * i;
-          w[i] = pack_bf16(ex2(x[j] + mneg), ex2(x[j + 1] + mneg));
-          l4[i] += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+          w[i] = pack2<T>(ex2(x[j] + mneg), ex2(x[j + 1] + mneg));
+          l4[i] += unpack_lo<T>(w[i]) + unpack_hi<T>(w[i]);
         }
         *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -481,11 +483,11 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
         const int dv0 = 256 * h + 128 * kh;   // this thread's 128 contiguous dv values of its row
         if (final_out) {
           uint4* dst = reinterpret_cast<uint4*>(
-              a.out + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + head) * 512 + dv0);
+              static_cast<uint16_t*>(a.out) + ((static_cast<size_t>(s.b) * a.s_q + srow) * a.h_q + head) * 512 + dv0);
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            dst[k] = make_uint4(pack_bf16(v[8 * k], v[8 * k + 1]), pack_bf16(v[8 * k + 2], v[8 * k + 3]),
-                                pack_bf16(v[8 * k + 4], v[8 * k + 5]), pack_bf16(v[8 * k + 6], v[8 * k + 7]));
+            dst[k] = make_uint4(pack2<T>(v[8 * k], v[8 * k + 1]), pack2<T>(v[8 * k + 2], v[8 * k + 3]),
+                                pack2<T>(v[8 * k + 4], v[8 * k + 5]), pack2<T>(v[8 * k + 6], v[8 * k + 7]));
         } else {
           float4* dst = reinterpret_cast<float4*>(
               a.o_part + ((static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + rr) * 512 + dv0);
@@ -506,6 +508,7 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
   }
 }
 
+template <int T>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -572,7 +575,7 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
   const uint32_t L_o_free = mapa_shared(smem_addr(&ct.o_free), 0);
 
   if (warp < 4) {
-    softmax_rows(a, ct, ps, tmem, ctl, rank, rb, g, md, L_s_free0, L_p_full0, L_o_free);
+    softmax_rows<T>(a, ct, ps, tmem, ctl, rank, rb, g, md, L_s_free0, L_p_full0, L_o_free);
   } else if (warp == 4) {
     score_loads(maps, a, ct, qs, ks, ctl, rank, rb, g, md, L_q_full, L_k_full0);
   } else if (warp == 5) {
@@ -580,7 +583,7 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
   } else {
     if (rank == 0 && (threadIdx.x & 31) == 0) {
       const bool pv_role = warp == 7;
-      (void)mma_issue(a, ct, qs, ps, ks, vs, tmem, ctl, md, pv_role);
+      (void)mma_issue<T>(a, ct, qs, ps, ks, vs, tmem, ctl, md, pv_role);
       // every MMA this thread issued has finished, and its commits have landed, before TMEM is
       // freed and the pair exits (the softmax has waited for them unless the pair is aborting)
       umma_commit_pair_leader(&ct.drain[pv_role ? 1 : 0]);
@@ -602,20 +605,27 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
 
 int decode_pair_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_decode_pair(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream) {
+template <int T>
+static cudaError_t launch_pair_t(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream) {
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(mla_decode_pair_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
   const int pairs = (row_blocks + 1) / 2;
   const dim3 grid(2 * pairs, a.h_kv, a.num_parts);
-  mla_decode_pair_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
+  mla_decode_pair_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_decode_pair(int dtype, const PairMaps& maps, const DecodeArgs& a, int row_blocks,
+                               cudaStream_t stream) {
+  if (dtype == kFP16) return launch_pair_t<kFP16>(maps, a, row_blocks, stream);
+  return launch_pair_t<kBF16>(maps, a, row_blocks, stream);
 }
 
 }  // namespace mla

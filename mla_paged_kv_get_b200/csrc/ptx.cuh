@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "../../include/mla_b200.h"
@@ -396,10 +397,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Element types of the path (q, cache, P, out).
+enum : int { kBF16 = MLA_DTYPE_BF16, kFP16 = MLA_DTYPE_FP16 };
+
+// tcgen05 instruction descriptor for kind::f16 with fp32 accumulation: A and B of type T.
+template <int T>
+__host__ __device__ constexpr uint32_t idesc_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                  // D format: f32
-         | (1u << 7)                                // A format: bf16
-         | (1u << 10)                               // B format: bf16
+         | ((T == kBF16 ? 1u : 0u) << 7)            // A format: bf16 (1) or f16 (0)
+         | ((T == kBF16 ? 1u : 0u) << 10)           // B format: bf16 (1) or f16 (0)
          | ((a_mn_major ? 1u : 0u) << 15)           // A major-ness
          | ((b_mn_major ? 1u : 0u) << 16)           // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
@@ -412,9 +418,35 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+// Two floats rounded to nearest-even values of type T, `lo` in the low half.
+template <int T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (T == kBF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// The two values of a pack2 word, back in fp32 (exact).
+template <int T>
+__device__ __forceinline__ float unpack_lo(uint32_t w) {
+  if constexpr (T == kBF16) return __uint_as_float(w << 16);
+  else return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+}
+template <int T>
+__device__ __forceinline__ float unpack_hi(uint32_t w) {
+  if constexpr (T == kBF16) return __uint_as_float(w & 0xffff0000u);
+  else return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+// One float rounded to nearest-even type T, as raw bits.
+template <int T>
+__device__ __forceinline__ uint16_t to_bits(float x) {
+  if constexpr (T == kBF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+  else return __half_as_ushort(__float2half_rn(x));
 }
 
 }  // namespace mla

@@ -9,7 +9,7 @@ Recipe (shapes follow the decode setting of the pages: bf16 paged latent
 cache, 64-token pages, one shared KV head of width 576, variable lengths):
 
 * ``q`` and the cache are float32 ``randn`` rounded to bf16 (round to
-  nearest even);
+  nearest even), or to fp16 for the fp16 path;
 * the used pages are ``randperm`` over all pages and dealt out in order to the
   page-table rows, so physical placement is shuffled;
 * one extra *poison page* filled with finite values of magnitude 30 sits in
@@ -71,8 +71,9 @@ def _gen(seed: int) -> torch.Generator:
 
 def build(name: str, seqlens, s_q: int, h_q: int, h_kv: int = 1, causal: bool = False,
           scale: float | None = None, seed: int = 0, shuffle: bool = True,
-          spare_slots: int = 1, poison: float = POISON) -> Workload:
-    """Lay out one workload with the recipe in the module docstring."""
+          spare_slots: int = 1, poison: float = POISON, dtype: torch.dtype = torch.bfloat16) -> Workload:
+    """Lay out one workload with the recipe in the module docstring (q and cache in `dtype`:
+    bf16, or fp16 for the fp16 path)."""
     g = _gen(seed)
     seqlens = torch.as_tensor(list(seqlens), dtype=torch.int32)
     B = seqlens.numel()
@@ -83,7 +84,7 @@ def build(name: str, seqlens, s_q: int, h_q: int, h_kv: int = 1, causal: bool = 
     poison_page = used                       # the last physical page
     num_pages = used + 1
 
-    q = torch.randn((B, s_q, h_q, D_QK), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    q = torch.randn((B, s_q, h_q, D_QK), generator=g, dtype=torch.float32).to(dtype)
     k = torch.randn((num_pages, PAGE, h_kv, D_QK), generator=g, dtype=torch.float32)
     sign = torch.randint(0, 2, (PAGE, h_kv, D_QK), generator=g, dtype=torch.int32) * 2 - 1
     k[poison_page] = poison * sign.float()
@@ -100,7 +101,7 @@ def build(name: str, seqlens, s_q: int, h_q: int, h_kv: int = 1, causal: bool = 
         if tail > 0:
             last = int(block_table[b, nb - 1])
             k[last, PAGE - tail:] = poison * sign[PAGE - tail:].float()
-    k_cache = k.to(torch.bfloat16)
+    k_cache = k.to(dtype)
     if scale is None:
         scale = D_QK ** -0.5
     return Workload(name, q, k_cache, block_table, seqlens, s_q, h_q, h_kv, causal,

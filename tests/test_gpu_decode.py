@@ -216,6 +216,20 @@ def test_step_replays_from_a_cuda_graph():
     del graph
 
 
+@pytest.mark.parametrize("shape", [(1, 16, False), (1, 32, False), (1, 64, False), (1, 128, False), (2, 64, True)])
+def test_fp16_inputs_match_oracle(shape):
+    """The fp16 path (same kernels, fp16 MMAs, P and out in fp16) against the oracle
+    on the fp16 inputs, split sequences included so the fp16 combine runs too."""
+    s_q, h_q, causal = shape
+    w = inputs.build(f"fp16_{s_q}x{h_q}", [1, 63, 64, 65, 200, 777, 2048], s_q=s_q, h_q=h_q, causal=causal,
+                     seed=61 + h_q, dtype=torch.float16)
+    o_ref, l_ref = oracle(w)
+    for sms in (148, 5):
+        out, lse, _, _ = run_gpu(w, num_sms=sms)
+        assert out.dtype == torch.float16
+        compare(w, out, lse, o_ref, l_ref, what=f"fp16 s_q={s_q} h_q={h_q} sms={sms}")
+
+
 # ---------------------------------------------------------------- failure paths
 
 def test_bounded_wait_reports_timeout_and_context_survives():
