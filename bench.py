@@ -422,7 +422,7 @@ def main(argv=None):
     roof.update({"traffic": traffic, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
                  if peak_src == "measured" else "fallback",
                  "kernel": ("mla_decode_pair_kernel" if R > 64 else "mla_decode_kernel")
-                 + " (CUDA events around its launch, every timed step)",
+                 + " (CUDA events around its launch on every fourth timed step)",
                  "combine_ms": combine_ms,
                  "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
                  "launch_ms": decode_ms,

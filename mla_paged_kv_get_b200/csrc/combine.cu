@@ -11,7 +11,8 @@
 //
 // One warp per query row: each lane owns 16 of the 512 values, reads them with
 // 16-byte loads per piece and writes 16 output values (two 16-byte stores), so a warp
-// moves whole 2 KB partial rows and a 1 KB output row.
+// moves whole 2 KB partial rows and a 1 KB output row; two pieces' loads are in
+// flight at once.
 #include "ptx.cuh"
 #include "decode.cuh"
 
@@ -26,6 +27,7 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restrict__ o_part,
                    const float* __restrict__ lse_part, uint16_t* __restrict__ out,
                    float* __restrict__ lse, int batch, int s_q, int h_q, int h_kv, int R) {
+  pdl_wait();   // the partials and piece counts come from the decode kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kRowsPerBlock + warp;
   const int g = blockIdx.y, b = blockIdx.z;
@@ -41,27 +43,45 @@ mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restri
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  const size_t row0 = (static_cast<size_t>(first) * h_kv + g) * R + r;   // piece i: row0 + i * h_kv * R
+  const size_t piece_stride = static_cast<size_t>(h_kv) * R;
   float top = -INFINITY;
-  for (int i = 0; i < n; ++i) {
-    top = fmaxf(top, __ldg(lse_part + (static_cast<size_t>(first + i) * h_kv + g) * R + r));
-  }
+  for (int i = 0; i < n; ++i) top = fmaxf(top, __ldg(lse_part + row0 + i * piece_stride));
   float total_lse = -INFINITY;
   if (top != -INFINITY) {
+    // Two pieces per step with both pieces' loads in flight before either is used.  A piece
+    // with lse = -inf saw no key; its row holds zeros (the decode kernel wrote it) and weighs 0.
     float wsum = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const size_t row = (static_cast<size_t>(first + i) * h_kv + g) * R + r;
-      const float li = __ldg(lse_part + row);
-      const float w = li == -INFINITY ? 0.f : expf(li - top);
-      wsum += w;
-      if (w != 0.f) {
-        const float4* src = reinterpret_cast<const float4*>(o_part + row * 512) + lane * 4;
+    for (int i = 0; i < n; i += 2) {
+      const bool two = i + 1 < n;
+      const size_t ra = row0 + i * piece_stride, rb = row0 + (i + (two ? 1 : 0)) * piece_stride;
+      const float la = __ldg(lse_part + ra), lb = two ? __ldg(lse_part + rb) : -INFINITY;
+      const float4* sa = reinterpret_cast<const float4*>(o_part + ra * 512) + lane * 4;
+      const float4* sb = reinterpret_cast<const float4*>(o_part + rb * 512) + lane * 4;
+      float4 xa[4], xb[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) xa[v] = __ldg(sa + v);
+      if (two) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) xb[v] = __ldg(sb + v);
+      }
+      const float wa = la == -INFINITY ? 0.f : expf(la - top);
+      const float wb = lb == -INFINITY ? 0.f : expf(lb - top);
+      wsum += wa + wb;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        acc[4 * v + 0] += wa * xa[v].x;
+        acc[4 * v + 1] += wa * xa[v].y;
+        acc[4 * v + 2] += wa * xa[v].z;
+        acc[4 * v + 3] += wa * xa[v].w;
+      }
+      if (two) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const float4 x = __ldg(src + v);
-          acc[4 * v + 0] += w * x.x;
-          acc[4 * v + 1] += w * x.y;
-          acc[4 * v + 2] += w * x.z;
-          acc[4 * v + 3] += w * x.w;
+          acc[4 * v + 0] += wb * xb[v].x;
+          acc[4 * v + 1] += wb * xb[v].y;
+          acc[4 * v + 2] += wb * xb[v].z;
+          acc[4 * v + 3] += wb * xb[v].w;
         }
       }
     }
@@ -89,12 +109,10 @@ cudaError_t launch_combine(int dtype, const int32_t* num_splits, const float* o_
   const dim3 grid((R + kRowsPerBlock - 1) / kRowsPerBlock, h_kv, batch);
   uint16_t* o = static_cast<uint16_t*>(out);
   if (dtype == kFP16)
-    mla_combine_kernel<kFP16><<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, o, lse, batch,
-                                                                     s_q, h_q, h_kv, R);
-  else
-    mla_combine_kernel<kBF16><<<grid, 32 * kRowsPerBlock, 0, stream>>>(num_splits, o_part, lse_part, o, lse, batch,
-                                                                     s_q, h_q, h_kv, R);
-  return cudaGetLastError();
+    return launch_pdl(mla_combine_kernel<kFP16>, grid, dim3(32 * kRowsPerBlock), 0, stream, num_splits, o_part,
+                      lse_part, o, lse, batch, s_q, h_q, h_kv, R);
+  return launch_pdl(mla_combine_kernel<kBF16>, grid, dim3(32 * kRowsPerBlock), 0, stream, num_splits, o_part,
+                    lse_part, o, lse, batch, s_q, h_q, h_kv, R);
 }
 
 }  // namespace mla

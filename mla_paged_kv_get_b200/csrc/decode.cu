@@ -66,8 +66,8 @@ struct Cfg {
   // same pages again, L2 hits).  A phase-parity wait is only sound when the waiter is at most
   // one phase ahead, so each ring has one consumer that takes it in order, and each slot one
   // producer warp (ring index modulo the producer count, ring sizes multiples of it).
-  static constexpr int kSlotsQk = N == 16 ? 8 : 4;
-  static constexpr int kSlotsPv = 4;
+  static constexpr int kSlotsQk = 4;
+  static constexpr int kSlotsPv = N == 16 ? 8 : 4;   // 16-row blocks: the value ring wants the depth (measured)
   static constexpr int kSlots = kSlotsQk + kSlotsPv;
   static_assert(kSlotsQk % kProducers == 0 && kSlotsPv % kProducers == 0, "slot ownership");
   static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
@@ -619,6 +619,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();   // the combine may start launching; it waits for this grid to finish
+  pdl_wait();      // the part table and piece counts come from the metadata kernel
   const uint32_t tmem = ct.tmem_base;
   const Ctl ctl{&ct.abort_flag, a.status, a.timeout_ns};
 
@@ -662,8 +664,7 @@ static cudaError_t launch_n(const CUtensorMap& tm_k, const CUtensorMap& tm_q, co
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  mla_decode_kernel<N, T><<<grid, Cfg<N>::kThreads, Cfg<N>::kSmemBytes, stream>>>(tm_k, tm_q, a);
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_kernel<N, T>, grid, dim3(Cfg<N>::kThreads), Cfg<N>::kSmemBytes, stream, tm_k, tm_q, a);
 }
 
 template <int T>

@@ -9,6 +9,24 @@
 
 namespace mla {
 
+// Launch with programmatic stream serialization: the kernel may begin (prologue up to its
+// pdl_wait()) while the previous kernel of the stream is still running.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 struct DecodeArgs {
   const uint8_t* k_cache;       // [num_pages, 64, h_kv, 576] bf16 (bytes, for L2 prefetch)
   const int32_t* block_table;   // [batch, max_pages]

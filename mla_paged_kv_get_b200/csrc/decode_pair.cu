@@ -564,6 +564,8 @@ mla_decode_pair_kernel(const __grid_constant__ PairMaps maps, const DecodeArgs a
   __syncthreads();
   cluster_sync();           // barriers of both CTAs initialised before any remote arrive or load
   tc_fence_after();
+  pdl_trigger();            // the combine may start launching; it waits for this grid to finish
+  pdl_wait();               // the part table and piece counts come from the metadata kernel
   const uint32_t tmem = ct.tmem_base;
   const Ctl ctl{&ct.abort_flag, a.status, a.timeout_ns};
   // barriers of the leader CTA, in the cluster shared window
@@ -618,8 +620,7 @@ static cudaError_t launch_pair_t(const PairMaps& maps, const DecodeArgs& a, int 
   }
   const int pairs = (row_blocks + 1) / 2;
   const dim3 grid(2 * pairs, a.h_kv, a.num_parts);
-  mla_decode_pair_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(maps, a);
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_pair_kernel<T>, grid, dim3(kThreads), kSmemBytes, stream, maps, a);
 }
 
 cudaError_t launch_decode_pair(int dtype, const PairMaps& maps, const DecodeArgs& a, int row_blocks,

@@ -68,6 +68,9 @@ struct Pos {
 __global__ void __launch_bounds__(kThreads, 1)
 mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_parts,
                     int32_t* __restrict__ tile_md, int32_t* __restrict__ num_splits) {
+  // The decode kernel, launched with programmatic serialization after this one, may start its
+  // prologue now; it reads tile_md and num_splits only after this grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ long long smem_ll[];
   long long* p_incl = smem_ll;                                        // [batch]  P_{b+1}
   int* n_s = reinterpret_cast<int*>(p_incl + batch);                  // [batch]  pages

@@ -397,6 +397,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start before the previous kernel in the stream has finished; pdl_wait() blocks until that
+// kernel has completed and its writes are visible (it returns at once otherwise), so it comes
+// before the first read of anything the previous kernel produces.  pdl_trigger() lets the next
+// kernel start launching early (it still waits for this one to complete in its own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Element types of the path (q, cache, P, out).
 enum : int { kBF16 = MLA_DTYPE_BF16, kFP16 = MLA_DTYPE_FP16 };
 
