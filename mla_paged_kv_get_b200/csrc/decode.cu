@@ -68,8 +68,11 @@ struct Cfg {
   // producer warp (ring index modulo the producer count, ring sizes multiples of it).
   static constexpr int kSlotsQk = 4;
   static constexpr int kSlotsPv = N == 16 ? 8 : 4;   // 16-row blocks: the value ring wants the depth (measured)
+  // 16-row blocks: two producer warps per ring, so a full ring never holds up the other's loads
+  static constexpr int kQkProducers = N == 16 ? 2 : kProducers;
+  static constexpr int kPvProducers = N == 16 ? 2 : kProducers;
   static constexpr int kSlots = kSlotsQk + kSlotsPv;
-  static_assert(kSlotsQk % kProducers == 0 && kSlotsPv % kProducers == 0, "slot ownership");
+  static_assert(kSlotsQk % kQkProducers == 0 && kSlotsPv % kPvProducers == 0, "slot ownership");
   static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
   static constexpr int kQBytes = N * 128 * 9;          // 9 chunks of [N rows][64 cols]
   static constexpr int kPBytes = kKeys * N * 2;        // P^T: [128 keys][N rows] bf16
@@ -121,9 +124,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ------------------------------------------------------------------ producers (warps 4 ..)
 // The slot-load sequence of a segment is fixed: Q, QK(0), then QK(t), PV(t-1) for t >= 1, then
 // PV(T-1); QK(t) is nine loads (one 64-column chunk of both pages), PV(t) eight (128 dv columns of
-// one page).  QK loads go to the score ring, PV loads to the value ring.  Producer warp w issues
-// the loads whose index in their ring is w modulo the number of producers, so it owns fixed
-// slots and waits only for the consumption of its own earlier loads.
+// one page).  QK loads go to the score ring, PV loads to the value ring.  Each ring has its set of
+// producer warps (all of them, or two per ring for 16-row blocks); a producer issues the loads whose
+// index in the ring is its own modulo the set's size, so it owns fixed slots and waits only for the
+// consumption of its own earlier loads.
 template <int N>
 __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, const DecodeArgs& a,
                               Ctrl& ct, uint8_t* slots, uint8_t* qs, const Ctl& ctl, int rb, int g,
@@ -185,7 +189,9 @@ __device__ void producer_role(const CUtensorMap* tm_k, const CUtensorMap* tm_q, 
     // one slot: two 8 KB boxes; returns false when the CTA is aborting
     auto issue = [&](bool pv, int chunk0, int chunk1, int pid0, int pid1) -> bool {
       const uint32_t ridx = pv ? pv_idx++ : qk_idx++;
-      if (static_cast<int>(ridx % C::kProducers) != pw) return true;
+      const int owner = pv ? C::kProducers - C::kPvProducers + static_cast<int>(ridx % C::kPvProducers)
+                           : static_cast<int>(ridx % C::kQkProducers);
+      if (owner != pw) return true;
       const uint32_t n = pv ? C::kSlotsPv : C::kSlotsQk;
       const uint32_t slot = (pv ? C::kSlotsQk : 0) + ridx % n;
       if (ridx >= n && !wait_uniform(&ct.empty[slot], ((ridx / n) - 1) & 1)) return false;
