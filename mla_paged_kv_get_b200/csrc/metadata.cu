@@ -8,14 +8,20 @@
 // partition of a cost line:
 //   sequence b with n_b = ceil(L_b / 64) pages occupies c_b = C + n_b units
 //   (0 if empty): C = 4 overhead units, then one unit per page.  P_b is the
-//   prefix sum of c_b, W = max(1, ceil(total / G)); part p owns units
-//   [p*W, (p+1)*W) (the last part everything after (G-1)*W), and page j of
-//   sequence b goes to the part that owns unit P_b + C + j.
+//   prefix sum of c_b.  Of the G_max table entries (the launch grid), G are
+//   used: with W(G) = max(1, ceil(total / G)), G in [ceil(G_max/2), G_max]
+//   minimises W(G) + S (S = 12 pages, the price of a merge pass) if some
+//   sequence's first and last page fall in different parts, else W(G); the
+//   largest G on ties; G = G_max when B * (number of candidates) > 32768 or
+//   total >= 2^31.
+//   W = W(G); part p < G owns units [p*W, (p+1)*W) (part G-1 everything after
+//   (G-1)*W), parts G .. G_max-1 are empty, and page j of sequence b goes to
+//   the part that owns unit P_b + C + j.
 //   pos(U) = first (sequence, page) whose unit is >= U, or (B, 0).  Entry p is
-//   (pos(p*W), pos((p+1)*W) or (B,0) for the last part, first_piece,
-//   n_pieces, 0, 0); a piece is a (part, sequence) pair with >= 1 page,
-//   numbered part by part; num_splits is the prefix sum of pieces per
-//   sequence.
+//   (pos(p*W), pos((p+1)*W) or (B,0) for part G-1, first_piece, n_pieces, 0,
+//   0), (B, 0, B, 0, total pieces, 0, 0, 0) for an empty part; a piece is a
+//   (part, sequence) pair with >= 1 page, numbered part by part; num_splits is
+//   the prefix sum of pieces per sequence.
 //
 // Every part and every sequence is independent given the prefix sums, so one
 // CTA does it with three block scans and one binary search per part: no
@@ -29,6 +35,8 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kOverhead = 4;
+constexpr int kSplitPenalty = 12;
+constexpr int kSearchBudget = 32768;   // (sequences x candidate part counts) examined at most
 constexpr int kMaxBatch = 8192;
 constexpr int kMaxParts = 4096;
 
@@ -83,13 +91,21 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   const int per = (batch + kThreads - 1) / kThreads;
   const int b0 = min(tid * per, batch), b1 = min(b0 + per, batch);
   long long my_cost = 0;
-  int my_ne = 0;
+  int my_ne = 0, my_max_n = 0;
   for (int b = b0; b < b1; ++b) {
     const int L = __ldg(seqlens + b);
     const int nb = L > 0 ? (L + 63) / 64 : 0;
     n_s[b] = nb;
     my_cost += nb > 0 ? nb + kOverhead : 0;
     my_ne += nb > 0;
+    my_max_n = max(my_max_n, nb);
+  }
+  __shared__ int max_n_w[kWarps];   // longest sequence (pages) per warp; published by the scan's barriers
+  {
+    int m = my_max_n;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) max_n_w[tid >> 5] = m;
   }
   long long total_cost, total_ne;
   long long run = block_exclusive_scan(my_cost, warp_buf, &total_cost);
@@ -104,7 +120,50 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   if (tid == 0) ne_s[batch] = static_cast<int>(total_ne);
   __syncthreads();
 
-  const long long G = num_parts;
+  // ---- number of parts in use
+  __shared__ unsigned long long best_key[kWarps];
+  int max_n = 0;
+  for (int w = 0; w < kWarps; ++w) max_n = max(max_n, max_n_w[w]);
+  const int g_lo = max(1, (num_parts + 1) / 2);
+  const int ncand = num_parts - g_lo + 1;
+  const long long w_max = total_cost > 0 ? (total_cost + num_parts - 1) / num_parts : 1;
+  int g_use = num_parts;
+  // Skipped when G_max must win anyway: a candidate that splits costs >= W(G_max) + S, one that does
+  // not must hold the longest sequence in one part (no part exceeds W units), so costs >= max_n; if
+  // max_n >= W(G_max) + S no candidate beats G_max, which wins the ties.  Otherwise only a G with
+  // max_n <= W(G) < W(G_max) + S can cost less than G_max, so only those (and G_max) are tested, one
+  // warp per candidate, in 32-bit integers (the cost line fits).
+  if (static_cast<long long>(batch) * ncand <= kSearchBudget && max_n < w_max + kSplitPenalty &&
+      total_cost < (1ll << 31)) {
+    const unsigned int total32 = static_cast<unsigned int>(total_cost);
+    const int warp = tid >> 5, lane = tid & 31;
+    unsigned long long key = ~0ull;   // smallest cost, then largest G: (cost << 32) | (~G & 0xffffffff)
+    for (int i = warp; i < ncand; i += kWarps) {
+      const unsigned int Gc = static_cast<unsigned int>(g_lo + i);
+      const unsigned int Wc = total32 > 0 ? (total32 + Gc - 1) / Gc : 1u;
+      const bool tested = static_cast<int>(Gc) == num_parts ||
+                          (Wc >= static_cast<unsigned int>(max_n) && Wc < static_cast<unsigned int>(w_max + kSplitPenalty));
+      if (!tested) continue;
+      bool split = false;
+      for (int b = lane; b < batch; b += 32) {
+        const int nb = n_s[b];
+        if (nb == 0) continue;
+        const unsigned int first = static_cast<unsigned int>((b > 0 ? p_incl[b - 1] : 0) + kOverhead);
+        const unsigned int pf = min(first / Wc, Gc - 1), pl = min((first + nb - 1) / Wc, Gc - 1);
+        split |= pf != pl;
+      }
+      split = __any_sync(0xffffffffu, split);
+      const unsigned long long cost = static_cast<unsigned long long>(Wc) + (split ? kSplitPenalty : 0);
+      const unsigned long long k2 = (cost << 32) | (0xffffffffull - static_cast<unsigned long long>(Gc));
+      key = k2 < key ? k2 : key;
+    }
+    if (lane == 0) best_key[warp] = key;
+    __syncthreads();
+    unsigned long long best = best_key[0];
+    for (int w = 1; w < kWarps; ++w) best = best_key[w] < best ? best_key[w] : best;
+    g_use = static_cast<int>(0xffffffffull - (best & 0xffffffffull));
+  }
+  const long long G = g_use;
   const long long W = total_cost > 0 ? (total_cost + G - 1) / G : 1;
 
   auto pos = [&](long long U) -> Pos {
@@ -125,8 +184,8 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
 
   // ---- parts: boundaries and piece counts
   for (int p = tid; p < num_parts; p += kThreads) {
-    const Pos be = pos(static_cast<long long>(p) * W);
-    const Pos en = p < num_parts - 1 ? pos(static_cast<long long>(p + 1) * W) : Pos{batch, 0};
+    const Pos be = p < G ? pos(static_cast<long long>(p) * W) : Pos{batch, 0};
+    const Pos en = p < G - 1 ? pos(static_cast<long long>(p + 1) * W) : Pos{batch, 0};
     const bool empty = be.b == en.b && be.page == en.page;
     np_s[p] = empty ? 0 : ne_s[en.b] - ne_s[be.b] + (en.page > 0 ? 1 : 0);
     int32_t* row = tile_md + static_cast<size_t>(p) * 8;

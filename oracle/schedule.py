@@ -12,18 +12,27 @@ this project's reading, stated in full in DESIGN.md ("Scheduler rule"):
 
 * rows per KV head ``R = s_q*h_q/h_kv`` are cut into row blocks of
   ``N = 16`` (R <= 16), ``32`` (R <= 32) or ``64`` rows; ``T = ceil(R/N)``;
-* ``G = max(1, num_sms // (h_kv*T))`` parts;
+* ``G_max = max(1, num_sms // (h_kv*T))`` parts at most (the launch grid);
 * the cost line: sequence ``b`` with ``n_b = ceil(L_b/64)`` pages occupies
   ``c_b = C + n_b`` units (0 if empty), ``C = 4`` units of per-sequence
   overhead first, then one unit per page; ``P_b`` is the prefix sum of the
   ``c_b`` and ``total = P_B``;
-* ``W = max(1, ceil(total / G))``; part ``p`` owns units ``[p*W, (p+1)*W)``,
-  the last part everything from ``(G-1)*W`` on;
+* the number of parts in use ``G`` is chosen among ``[ceil(G_max/2), G_max]``:
+  with ``W(G) = max(1, ceil(total / G))``, sequence ``b`` is *split* by ``G``
+  when its first and last page fall in different parts
+  (``min(unit // W, G-1)`` differs for ``P_b + C`` and ``P_b + C + n_b - 1``);
+  ``cost(G) = W(G) + S`` if any sequence is split, else ``W(G)``, with
+  ``S = 12`` pages (a split costs the merge pass); ``G`` minimises the cost,
+  the largest ``G`` on ties.  When ``B * (number of candidates)`` exceeds
+  32768, or ``total >= 2**31``, the search is skipped and ``G = G_max``;
+* ``W = W(G)``; part ``p < G`` owns units ``[p*W, (p+1)*W)``, part ``G-1``
+  everything from ``(G-1)*W`` on, and parts ``G .. G_max-1`` are empty;
 * page ``j`` of sequence ``b`` goes to the part owning unit ``P_b + C + j``;
 * ``pos(U)``: the first (sequence, page) whose unit is ``>= U`` (``(B, 0)``
   past the end); ``tile_md[p] = (begin_b, begin_page, end_b, end_page,
   first_piece, n_pieces, 0, 0)`` with ``begin = pos(p*W)`` and
-  ``end = pos((p+1)*W)`` (``(B, 0)`` for the last part), end exclusive;
+  ``end = pos((p+1)*W)`` (``(B, 0)`` for part ``G-1``), end exclusive; an
+  empty part ``p >= G`` is ``(B, 0, B, 0, total pieces, 0, 0, 0)``;
 * a piece is a (part, sequence) pair with at least one page; pieces are
   numbered part by part, sequences in order within a part; ``first_piece``
   is the number of pieces in earlier parts; ``num_splits`` is the prefix sum
@@ -35,6 +44,8 @@ No floating point anywhere.
 from __future__ import annotations
 
 SPLIT_OVERHEAD_PAGES = 4   # C
+SPLIT_PENALTY_PAGES = 12   # S
+SEARCH_BUDGET = 32768      # (sequences x candidate part counts) examined at most
 PAGE = 64
 MD_WORDS = 8
 
@@ -60,18 +71,42 @@ def _pages(seqlens):
     return [(int(L) + PAGE - 1) // PAGE if int(L) > 0 else 0 for L in seqlens]
 
 
+def parts_in_use(n, start, total, G_max: int) -> int:
+    """The number of parts G the rule picks (see the module docstring)."""
+    C, S = SPLIT_OVERHEAD_PAGES, SPLIT_PENALTY_PAGES
+    lo = max(1, (G_max + 1) // 2)
+    if len(n) * (G_max - lo + 1) > SEARCH_BUDGET or total >= 1 << 31:
+        return G_max
+    best_cost, best_G = None, G_max
+    for G in range(lo, G_max + 1):
+        W = max(1, (total + G - 1) // G)
+        split = False
+        for b in range(len(n)):
+            if n[b] > 0:
+                first = start[b] + C
+                last = first + n[b] - 1
+                if min(first // W, G - 1) != min(last // W, G - 1):
+                    split = True
+                    break
+        cost = W + (S if split else 0)
+        if best_cost is None or cost <= best_cost:
+            best_cost, best_G = cost, G
+    return best_G
+
+
 def get_metadata(seqlens, rows_per_kv: int, h_kv: int, num_sms: int):
     """Return ``(tile_md, num_splits)`` as lists of Python ints."""
     C = SPLIT_OVERHEAD_PAGES
     n = _pages(seqlens)
     B = len(n)
-    G = num_parts(rows_per_kv, h_kv, num_sms)
+    G_max = num_parts(rows_per_kv, h_kv, num_sms)
     start = []          # P_b
     acc = 0
     for nb in n:
         start.append(acc)
         acc += nb + C if nb > 0 else 0
     total = acc
+    G = parts_in_use(n, start, total, G_max)
     W = max(1, (total + G - 1) // G)
 
     def part_of(unit):
@@ -97,6 +132,8 @@ def get_metadata(seqlens, rows_per_kv: int, h_kv: int, num_sms: int):
         pieces = sorted({b for (b, j), q in owner.items() if q == p})
         tile_md.append([begin[0], begin[1], end[0], end[1], first, len(pieces), 0, 0])
         first += len(pieces)
+    for p in range(G, G_max):
+        tile_md.append([B, 0, B, 0, first, 0, 0, 0])
 
     num_splits = [0]
     for b in range(B):

@@ -21,13 +21,22 @@ def test_hand_worked_cases():
 
 def check_invariants(seqlens, rows_per_kv, h_kv, num_sms):
     md, ns = sch.get_metadata(seqlens, rows_per_kv, h_kv, num_sms)
-    G = sch.num_parts(rows_per_kv, h_kv, num_sms)
+    G_max = sch.num_parts(rows_per_kv, h_kv, num_sms)
     B = len(seqlens)
     C = sch.SPLIT_OVERHEAD_PAGES
     n = [(L + 63) // 64 for L in seqlens]
     total = sum(x + C for x in n if x > 0)
+    # the parts in use (the choice itself is pinned by the hand cases and the equal-length case)
+    starts = []
+    acc = 0
+    for x in n:
+        starts.append(acc)
+        acc += x + C if x > 0 else 0
+    G = sch.parts_in_use(n, starts, total, G_max)
+    assert (G_max + 1) // 2 <= G <= G_max
+    assert all(md[p] == [B, 0, B, 0, md[p][4], 0, 0, 0] for p in range(G, G_max))
     W = max(1, (total + G - 1) // G)
-    assert len(md) == G and len(ns) == B + 1 and ns[0] == 0
+    assert len(md) == G_max and len(ns) == B + 1 and ns[0] == 0
     covered = {}
     pieces_seen = [0] * B
     prev_end = (0, 0)
@@ -82,6 +91,18 @@ def test_all_empty_and_single_token():
     assert ns == [0, 0, 0, 0]
     md, ns = check_invariants([1], 128, 1, 148)
     assert ns == [0, 1]
+
+
+def test_equal_lengths_take_one_part_each():
+    """64 sequences of 64 pages (68 units each) and at most 74 parts: 64 parts of 68 units
+    hold one whole sequence each (cost 68), while any 65..74 parts are narrower than a
+    sequence's 64 pages at some boundary and split one (cost >= 60 + 12); so 64 parts are
+    used, each sequence is one piece, and parts 64..73 are empty."""
+    lens = [4096] * 64
+    md, ns = check_invariants(lens, 128, 1, 148)
+    assert ns == list(range(65))
+    assert all(md[p][:6] == [p, 0, p + 1, 0, p, 1] for p in range(64))
+    assert all(md[p] == [64, 0, 64, 0, 64, 0, 0, 0] for p in range(64, 74))
 
 
 def test_long_sequences_get_split():
