@@ -114,32 +114,6 @@ __device__ __forceinline__ bool drain_phase(uint64_t* bar, uint32_t parity, uint
   return true;
 }
 
-// Wait on a barrier that threads of the peer CTA arrive on remotely. The
-// data those arrivals publish is read by the tensor cores of the CTA that
-// wrote it (its half of a paired MMA operand) and was fenced into the async
-// proxy before the arrive, so the default-scope test suffices.
-__device__ __forceinline__ bool mbar_test_cluster(uint64_t* bar, uint32_t parity) {
-  return mbar_test(bar, parity);
-}
-
-__device__ __forceinline__ bool wait_phase_cluster(uint64_t* bar, uint32_t parity, const Ctl& c) {
-  if (mbar_test_cluster(bar, parity)) return true;
-  uint64_t t0 = 0;
-  for (uint32_t polls = 1;; ++polls) {
-    if (mbar_test_cluster(bar, parity)) return true;
-    if ((polls & 255u) == 0) {
-      if (*c.abort_flag) return false;
-      const uint64_t now = global_timer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > c.timeout_ns) {
-        raise_abort(c, MLA_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -167,17 +141,9 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// TMA tile load into this CTA's shared memory whose completion is counted on
-// a barrier of either CTA of the pair (cluster address `bar_cluster`).
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
-                                                 int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
+// TMA tile loads into this CTA's shared memory.  The _pair forms (cta_group::2) count their completion
+// on a barrier of either CTA of the pair (cluster address `bar_cluster`); the others on this CTA's `bar`.
+// None uses cluster multicast: each CTA loads its own tiles.
 __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
                                                  int c0, int c1, int c2, int c3) {
   asm volatile(
@@ -219,16 +185,6 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)),
-        "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(
@@ -257,16 +213,6 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
       ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2),
         "r"(c3), "r"(c4)
       : "memory");
-}
-
-// One 128-byte line into L2 (load/store unit path, does not occupy the TMA unit).
-__device__ __forceinline__ void l2_prefetch_line(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// Pull `bytes` (a multiple of 16) starting at `src` into L2 without using shared memory.
-__device__ __forceinline__ void l2_prefetch(const void* src, size_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(static_cast<uint32_t>(bytes)) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
