@@ -80,11 +80,16 @@ def load_traffic(workload: str):
     return None, None
 
 
+# the files the decode kernels (and the tensor maps they are launched with) are built from
+DECODE_SOURCES = ("capi.cu", "decode.cu", "decode.cuh", "decode_pair.cu", "ptx.cuh", "segments.cuh")
+
+
 def source_sha() -> str:
+    """Hash of the decode kernels' sources: stored ncu counters apply only while it is unchanged."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_paged_kv_get_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in DECODE_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())

@@ -60,6 +60,25 @@ def test_metadata_bit_exact(seed):
         assert ns.cpu().tolist() == ns_ref
 
 
+
+@pytest.mark.parametrize("rows,sms", [(128, 148), (16, 148), (128, 20)])
+def test_metadata_part_count_search_bit_exact(rows, sms):
+    """Near-equal batches around the part limit, where the part-count search
+    runs and sometimes leaves trailing parts empty."""
+    g = torch.Generator().manual_seed(rows * 1000 + sms)
+    G_max = sch.num_parts(rows, 1, sms)
+    fewer = 0
+    for B in [G_max // 2, G_max // 2 + 1, G_max - 1, G_max, G_max + 1, 2 * G_max - 3, 3 * G_max]:
+        for jitter in [0, 64, 700]:
+            lens = 4096 + torch.randint(0, jitter + 1, (B,), generator=g)
+            md, ns = binding.get_metadata(lens.to(torch.int32).cuda(), rows, 1, sms)
+            md_ref, ns_ref = sch.get_metadata(lens.tolist(), rows, 1, sms)
+            assert md.cpu().tolist() == md_ref, (B, jitter)
+            assert ns.cpu().tolist() == ns_ref, (B, jitter)
+            fewer += md_ref[-1][:4] == [B, 0, B, 0]
+    assert fewer > 0   # the cases do reach a part count below the limit
+
+
 # ---------------------------------------------------------------- decode parity
 
 def test_tiny_config():
