@@ -27,7 +27,8 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restrict__ o_part,
                    const float* __restrict__ lse_part, uint16_t* __restrict__ out,
                    float* __restrict__ lse, int batch, int s_q, int h_q, int h_kv, int R) {
-  pdl_wait();   // the partials and piece counts come from the decode kernel
+  pdl_trigger();   // the next kernel (a later step's metadata) may start launching; it waits for this grid
+  pdl_wait();      // the partials and piece counts come from the decode kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kRowsPerBlock + warp;
   const int g = blockIdx.y, b = blockIdx.z;

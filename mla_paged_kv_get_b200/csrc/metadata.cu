@@ -24,8 +24,11 @@
 //   the prefix sum of pieces per sequence.
 //
 // Every part and every sequence is independent given the prefix sums, so one
-// CTA does it with three block scans and one binary search per part: no
-// sequential sweep.
+// CTA does it with two block scans (cost, then pieces) and one binary search
+// per part boundary: no sequential sweep.  Because a sequence's pieces lie in
+// consecutive parts, numbering pieces part by part is the same as numbering
+// them sequence by sequence, so a part's first piece follows from num_splits
+// in closed form.
 #include "decode.cuh"
 
 namespace mla {
@@ -34,6 +37,7 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+static_assert(kWarps == 32, "per-warp partials are reduced by one warp, one per lane");
 constexpr int kOverhead = 4;
 constexpr int kSplitPenalty = 12;
 constexpr int kSearchBudget = 32768;   // (sequences x candidate part counts) examined at most
@@ -79,25 +83,26 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   // The decode kernel, launched with programmatic serialization after this one, may start its
   // prologue now; it reads tile_md and num_splits only after this grid has completed.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // This grid may itself start before the previous kernel of the stream has finished (the combine
+  // of an earlier step still reads num_splits): wait for it before reading or writing anything.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ long long smem_ll[];
   long long* p_incl = smem_ll;                                        // [batch]  P_{b+1}
   int* n_s = reinterpret_cast<int*>(p_incl + batch);                  // [batch]  pages
-  int* ne_s = n_s + batch;                                            // [batch+1] non-empty before b
-  int* np_s = ne_s + batch + 1;                                       // [num_parts] pieces per part
+  int* ns_s = n_s + batch;                                            // [batch+1] num_splits
   __shared__ long long warp_buf[33];
   const int tid = threadIdx.x;
 
-  // ---- prefix sums of cost and of non-empty sequences (contiguous chunk per thread)
+  // ---- prefix sums of cost (contiguous chunk of sequences per thread)
   const int per = (batch + kThreads - 1) / kThreads;
   const int b0 = min(tid * per, batch), b1 = min(b0 + per, batch);
   long long my_cost = 0;
-  int my_ne = 0, my_max_n = 0;
+  int my_max_n = 0;
   for (int b = b0; b < b1; ++b) {
     const int L = __ldg(seqlens + b);
     const int nb = L > 0 ? (L + 63) / 64 : 0;
     n_s[b] = nb;
     my_cost += nb > 0 ? nb + kOverhead : 0;
-    my_ne += nb > 0;
     my_max_n = max(my_max_n, nb);
   }
   __shared__ int max_n_w[kWarps];   // longest sequence (pages) per warp; published by the scan's barriers
@@ -107,23 +112,21 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((tid & 31) == 0) max_n_w[tid >> 5] = m;
   }
-  long long total_cost, total_ne;
+  long long total_cost;
   long long run = block_exclusive_scan(my_cost, warp_buf, &total_cost);
-  long long run_ne = block_exclusive_scan(my_ne, warp_buf, &total_ne);
   for (int b = b0; b < b1; ++b) {
     const int nb = n_s[b];
-    ne_s[b] = static_cast<int>(run_ne);
     run += nb > 0 ? nb + kOverhead : 0;
-    run_ne += nb > 0;
     p_incl[b] = run;
   }
-  if (tid == 0) ne_s[batch] = static_cast<int>(total_ne);
   __syncthreads();
 
   // ---- number of parts in use
   __shared__ unsigned long long best_key[kWarps];
-  int max_n = 0;
-  for (int w = 0; w < kWarps; ++w) max_n = max(max_n, max_n_w[w]);
+  const int lane = tid & 31;
+  int max_n = max_n_w[lane];   // kWarps == 32: one warp entry per lane
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) max_n = max(max_n, __shfl_xor_sync(0xffffffffu, max_n, o));
   const int g_lo = max(1, (num_parts + 1) / 2);
   const int ncand = num_parts - g_lo + 1;
   const long long w_max = total_cost > 0 ? (total_cost + num_parts - 1) / num_parts : 1;
@@ -136,7 +139,7 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   if (static_cast<long long>(batch) * ncand <= kSearchBudget && max_n < w_max + kSplitPenalty &&
       total_cost < (1ll << 31)) {
     const unsigned int total32 = static_cast<unsigned int>(total_cost);
-    const int warp = tid >> 5, lane = tid & 31;
+    const int warp = tid >> 5;
     unsigned long long key = ~0ull;   // smallest cost, then largest G: (cost << 32) | (~G & 0xffffffff)
     for (int i = warp; i < ncand; i += kWarps) {
       const unsigned int Gc = static_cast<unsigned int>(g_lo + i);
@@ -159,12 +162,22 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
     }
     if (lane == 0) best_key[warp] = key;
     __syncthreads();
-    unsigned long long best = best_key[0];
-    for (int w = 1; w < kWarps; ++w) best = best_key[w] < best ? best_key[w] : best;
+    unsigned long long best = best_key[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+      best = y < best ? y : best;
+    }
     g_use = static_cast<int>(0xffffffffull - (best & 0xffffffffull));
   }
+  // Quotients on the cost line in 32 bits whenever it fits (the usual case): a 64-bit division is
+  // a long software sequence on the GPU.
+  const bool line32 = total_cost < (1ll << 31);
+  auto udiv = [line32](long long n, long long d) -> long long {
+    return line32 ? static_cast<long long>(static_cast<unsigned int>(n) / static_cast<unsigned int>(d)) : n / d;
+  };
   const long long G = g_use;
-  const long long W = total_cost > 0 ? (total_cost + G - 1) / G : 1;
+  const long long W = total_cost > 0 ? udiv(total_cost + G - 1, G) : 1;
 
   auto pos = [&](long long U) -> Pos {
     if (U >= total_cost) return Pos{batch, 0};
@@ -178,58 +191,51 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
     return Pos{lo, pg > 0 ? static_cast<int>(pg) : 0};
   };
   auto part_of = [&](long long unit) -> int {
-    const long long p = unit / W;
+    const long long p = udiv(unit, W);
     return static_cast<int>(p < G - 1 ? p : G - 1);
   };
+  auto first_unit = [&](int b) -> long long { return (b > 0 ? p_incl[b - 1] : 0) + kOverhead; };
 
-  // ---- parts: boundaries and piece counts
-  for (int p = tid; p < num_parts; p += kThreads) {
-    const Pos be = p < G ? pos(static_cast<long long>(p) * W) : Pos{batch, 0};
-    const Pos en = p < G - 1 ? pos(static_cast<long long>(p + 1) * W) : Pos{batch, 0};
-    const bool empty = be.b == en.b && be.page == en.page;
-    np_s[p] = empty ? 0 : ne_s[en.b] - ne_s[be.b] + (en.page > 0 ? 1 : 0);
-    int32_t* row = tile_md + static_cast<size_t>(p) * 8;
-    row[0] = be.b;
-    row[1] = be.page;
-    row[2] = en.b;
-    row[3] = en.page;
-    row[6] = 0;
-    row[7] = 0;
-  }
-
-  // ---- pieces per sequence -> num_splits
+  // ---- pieces per sequence -> num_splits (a sequence's pieces sit in consecutive parts)
   long long my_pieces = 0;
   for (int b = b0; b < b1; ++b) {
     const int nb = n_s[b];
-    if (nb > 0) {
-      const long long first_unit = (b > 0 ? p_incl[b - 1] : 0) + kOverhead;
-      my_pieces += part_of(first_unit + nb - 1) - part_of(first_unit) + 1;
-    }
+    if (nb > 0) my_pieces += part_of(first_unit(b) + nb - 1) - part_of(first_unit(b)) + 1;
   }
   long long total_pieces;
   long long run_p = block_exclusive_scan(my_pieces, warp_buf, &total_pieces);
   for (int b = b0; b < b1; ++b) {
     num_splits[b] = static_cast<int32_t>(run_p);
+    ns_s[b] = static_cast<int>(run_p);
     const int nb = n_s[b];
-    if (nb > 0) {
-      const long long first_unit = (b > 0 ? p_incl[b - 1] : 0) + kOverhead;
-      run_p += part_of(first_unit + nb - 1) - part_of(first_unit) + 1;
-    }
+    if (nb > 0) run_p += part_of(first_unit(b) + nb - 1) - part_of(first_unit(b)) + 1;
   }
-  if (tid == 0) num_splits[batch] = static_cast<int32_t>(total_pieces);
+  if (tid == 0) {
+    num_splits[batch] = static_cast<int32_t>(total_pieces);
+    ns_s[batch] = static_cast<int>(total_pieces);
+  }
+  __syncthreads();
 
-  // ---- first piece of each part: prefix over parts (contiguous chunk per thread)
-  const int pper = (num_parts + kThreads - 1) / kThreads;
-  const int p0 = min(tid * pper, num_parts), p1 = min(p0 + pper, num_parts);
-  long long my_np = 0;
-  for (int p = p0; p < p1; ++p) my_np += np_s[p];
-  long long total_np;
-  long long run_np = block_exclusive_scan(my_np, warp_buf, &total_np);
-  for (int p = p0; p < p1; ++p) {
+  // ---- parts.  Pieces are numbered part by part, which along the cost line is also sequence by
+  // sequence, so the pieces before the part that begins at `be` are those of the sequences before
+  // be.b plus, when be cuts sequence be.b, one per part from the one holding its page 0 to this one.
+  auto pieces_before = [&](int p, Pos be) -> int {
+    return ns_s[be.b] + (be.page > 0 ? p - part_of(first_unit(be.b)) : 0);
+  };
+  for (int p = tid; p < num_parts; p += kThreads) {
+    const Pos be = p < G ? pos(static_cast<long long>(p) * W) : Pos{batch, 0};
+    const Pos en = p < G - 1 ? pos(static_cast<long long>(p + 1) * W) : Pos{batch, 0};
+    const int first = pieces_before(p, be);
+    const int next = p < G - 1 ? pieces_before(p + 1, en) : ns_s[batch];
     int32_t* row = tile_md + static_cast<size_t>(p) * 8;
-    row[4] = static_cast<int32_t>(run_np);
-    row[5] = np_s[p];
-    run_np += np_s[p];
+    row[0] = be.b;
+    row[1] = be.page;
+    row[2] = en.b;
+    row[3] = en.page;
+    row[4] = first;
+    row[5] = next - first;
+    row[6] = 0;
+    row[7] = 0;
   }
 }
 
@@ -240,20 +246,19 @@ int metadata_max_parts() { return kMaxParts; }
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,
                             int32_t* num_splits, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(batch) * sizeof(long long) + (2 * batch + 1) * sizeof(int) +
-                      static_cast<size_t>(num_parts) * sizeof(int);
+  const size_t smem = static_cast<size_t>(batch) * sizeof(long long) + (2 * batch + 1) * sizeof(int);
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
     const int max_smem = kMaxBatch * static_cast<int>(sizeof(long long)) +
-                         (2 * kMaxBatch + 1) * static_cast<int>(sizeof(int)) + kMaxParts * static_cast<int>(sizeof(int));
+                         (2 * kMaxBatch + 1) * static_cast<int>(sizeof(int));
     cudaError_t e = cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  mla_metadata_kernel<<<1, kThreads, smem, stream>>>(seqlens, batch, num_parts, tile_md, num_splits);
-  return cudaGetLastError();
+  return launch_pdl(mla_metadata_kernel, dim3(1), dim3(kThreads), smem, stream, seqlens, batch, num_parts, tile_md,
+                    num_splits);
 }
 
 }  // namespace mla
