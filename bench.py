@@ -351,9 +351,10 @@ def main(argv=None):
     assert int(status.item()) == 0, binding.status_string(int(status.item()))
 
     # ---- timed region: K steps, barrier + sync on both sides.  Every EV_EVERY-th step carries
-    # events around the decode and combine launches (on the launching stream); events on every
-    # step would add their own gaps to the step time.
-    EV_EVERY = 4
+    # events around the decode and combine launches (on the launching stream).  An event between
+    # two launches breaks their programmatic-launch overlap, so the instrumented steps are slower
+    # than the rest: they are kept few (500 steps -> 32 samples of each kernel).
+    EV_EVERY = 16
     n_ev = min((args.steps + EV_EVERY - 1) // EV_EVERY, 512)
     evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_ev)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -427,7 +428,7 @@ def main(argv=None):
     roof.update({"traffic": traffic, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
                  if peak_src == "measured" else "fallback",
                  "kernel": ("mla_decode_pair_kernel" if R > 64 else "mla_decode_kernel")
-                 + " (CUDA events around its launch on every fourth timed step)",
+                 + f" (CUDA events around its launch on every {EV_EVERY}th timed step)",
                  "combine_ms": combine_ms,
                  "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
                  "launch_ms": decode_ms,
