@@ -79,6 +79,23 @@ def test_metadata_part_count_search_bit_exact(rows, sms):
     assert fewer > 0   # the cases do reach a part count below the limit
 
 
+
+def test_metadata_max_batch_bit_exact():
+    """The largest batch the metadata call accepts (8192 sequences: the kernel's shared-memory
+    tables are at their largest), with empty sequences mixed in; one more is rejected."""
+    g = torch.Generator().manual_seed(8192)
+    B = 8192
+    lens = torch.randint(0, 2049, (B,), generator=g)
+    lens[::7] = 0
+    for rows, sms in [(16, 148), (128, 148)]:
+        md, ns = binding.get_metadata(lens.to(torch.int32).cuda(), rows, 1, sms)
+        md_ref, ns_ref = sch.get_metadata(lens.tolist(), rows, 1, sms)
+        assert md.cpu().tolist() == md_ref
+        assert ns.cpu().tolist() == ns_ref
+    with pytest.raises(binding.MLAError):
+        binding.get_metadata(torch.ones(B + 1, dtype=torch.int32, device="cuda"), 16, 1, 148)
+
+
 # ---------------------------------------------------------------- decode parity
 
 def test_tiny_config():
