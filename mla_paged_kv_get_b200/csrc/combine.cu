@@ -11,8 +11,9 @@
 //
 // One warp per query row: each lane owns 16 of the 512 values, reads them with
 // 16-byte loads per piece and writes 16 output values (two 16-byte stores), so a warp
-// moves whole 2 KB partial rows and a 1 KB output row; two pieces' loads are in
-// flight at once.
+// moves whole 2 KB partial rows and a 1 KB output row.  The lse values of all pieces
+// are read in one round trip (one per lane) and four pieces' rows are in flight at
+// once, so a row split n ways costs about 1 + n/4 memory latencies.
 #include "ptx.cuh"
 #include "decode.cuh"
 
@@ -21,6 +22,7 @@ namespace mla {
 namespace {
 
 constexpr int kRowsPerBlock = 4;
+constexpr int kPiecesInFlight = 4;   // O rows of four pieces loaded before any is used
 
 template <int T>
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
@@ -46,46 +48,52 @@ mla_combine_kernel(const int32_t* __restrict__ num_splits, const float* __restri
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   const size_t row0 = (static_cast<size_t>(first) * h_kv + g) * R + r;   // piece i: row0 + i * h_kv * R
   const size_t piece_stride = static_cast<size_t>(h_kv) * R;
+  // The lse of every piece at once, lane i holding pieces i, i + 32, ...: one memory round trip.
   float top = -INFINITY;
-  for (int i = 0; i < n; ++i) top = fmaxf(top, __ldg(lse_part + row0 + i * piece_stride));
+  for (int i = lane; i < n; i += 32) top = fmaxf(top, __ldg(lse_part + row0 + i * piece_stride));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) top = fmaxf(top, __shfl_xor_sync(0xffffffffu, top, o));
   float total_lse = -INFINITY;
   if (top != -INFINITY) {
-    // Two pieces per step with both pieces' loads in flight before either is used.  A piece
-    // with lse = -inf saw no key; its row holds zeros (the decode kernel wrote it) and weighs 0.
-    float wsum = 0.f;
-    for (int i = 0; i < n; i += 2) {
-      const bool two = i + 1 < n;
-      const size_t ra = row0 + i * piece_stride, rb = row0 + (i + (two ? 1 : 0)) * piece_stride;
-      const float la = __ldg(lse_part + ra), lb = two ? __ldg(lse_part + rb) : -INFINITY;
-      const float4* sa = reinterpret_cast<const float4*>(o_part + ra * 512) + lane * 4;
-      const float4* sb = reinterpret_cast<const float4*>(o_part + rb * 512) + lane * 4;
-      float4 xa[4], xb[4];
+    // Pieces 32 at a time: lane i holds the weight of piece base + i; their O rows are read four
+    // pieces at a time, all four in flight before any is used.  A piece with lse = -inf saw no key;
+    // its row holds zeros (the decode kernel wrote it) and weighs 0.
+    float wpart = 0.f;
+    for (int base = 0; base < n; base += 32) {
+      const int mine = base + lane;
+      const float li = mine < n ? __ldg(lse_part + row0 + mine * piece_stride) : -INFINITY;
+      const float wi = li == -INFINITY ? 0.f : expf(li - top);
+      wpart += wi;
+      const int cnt = min(32, n - base);
+      for (int j = 0; j < cnt; j += kPiecesInFlight) {
+        float4 x[kPiecesInFlight][4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) xa[v] = __ldg(sa + v);
-      if (two) {
+        for (int k = 0; k < kPiecesInFlight; ++k) {
+          if (j + k < cnt) {
+            const float4* src =
+                reinterpret_cast<const float4*>(o_part + (row0 + (base + j + k) * piece_stride) * 512) + lane * 4;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) xb[v] = __ldg(sb + v);
-      }
-      const float wa = la == -INFINITY ? 0.f : expf(la - top);
-      const float wb = lb == -INFINITY ? 0.f : expf(lb - top);
-      wsum += wa + wb;
+            for (int v = 0; v < 4; ++v) x[k][v] = __ldg(src + v);
+          }
+        }
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        acc[4 * v + 0] += wa * xa[v].x;
-        acc[4 * v + 1] += wa * xa[v].y;
-        acc[4 * v + 2] += wa * xa[v].z;
-        acc[4 * v + 3] += wa * xa[v].w;
-      }
-      if (two) {
+        for (int k = 0; k < kPiecesInFlight; ++k) {
+          const float w = __shfl_sync(0xffffffffu, wi, (j + k) & 31);
+          if (j + k < cnt) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          acc[4 * v + 0] += wb * xb[v].x;
-          acc[4 * v + 1] += wb * xb[v].y;
-          acc[4 * v + 2] += wb * xb[v].z;
-          acc[4 * v + 3] += wb * xb[v].w;
+            for (int v = 0; v < 4; ++v) {
+              acc[4 * v + 0] += w * x[k][v].x;
+              acc[4 * v + 1] += w * x[k][v].y;
+              acc[4 * v + 2] += w * x[k][v].z;
+              acc[4 * v + 3] += w * x[k][v].w;
+            }
+          }
         }
       }
     }
+    float wsum = wpart;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     const float inv = 1.f / wsum;
 #pragma unroll
     for (int i = 0; i < 16; ++i) acc[i] *= inv;
