@@ -66,11 +66,14 @@ struct Cfg {
   // same pages again, L2 hits).  A phase-parity wait is only sound when the waiter is at most
   // one phase ahead, so each ring has one consumer that takes it in order, and each slot one
   // producer warp (ring index modulo the producer count, ring sizes multiples of it).
-  static constexpr int kSlotsQk = 4;
-  static constexpr int kSlotsPv = N == 16 ? 8 : 4;   // 16-row blocks: the value ring wants the depth (measured)
-  // 16-row blocks: two producer warps per ring, so a full ring never holds up the other's loads
-  static constexpr int kQkProducers = N == 16 ? 2 : kProducers;
-  static constexpr int kPvProducers = N == 16 ? 2 : kProducers;
+  // 16-row blocks (measured): the score ring streams from HBM and is held by how fast its loads
+  // are issued, so it gets three producer warps and six slots; the value ring's loads hit L2 and
+  // one warp keeps up, but it needs six slots (four cost 30 %).  The rings are disjoint, so a full
+  // one never holds up the other's loads.
+  static constexpr int kSlotsQk = N == 16 ? 6 : 4;
+  static constexpr int kSlotsPv = N == 16 ? 6 : 4;
+  static constexpr int kQkProducers = N == 16 ? 3 : kProducers;
+  static constexpr int kPvProducers = N == 16 ? 1 : kProducers;
   static constexpr int kSlots = kSlotsQk + kSlotsPv;
   static_assert(kSlotsQk % kQkProducers == 0 && kSlotsPv % kPvProducers == 0, "slot ownership");
   static constexpr int kPBuf = N == 64 ? 1 : 2;        // P^T buffers (one for N = 64: smem goes to the ring)
