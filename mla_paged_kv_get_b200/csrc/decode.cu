@@ -664,15 +664,9 @@ int decode_smem_bytes(int n) {
 template <int N, int T>
 static cudaError_t launch_n(const CUtensorMap& tm_k, const CUtensorMap& tm_q, const DecodeArgs& a, dim3 grid,
                             cudaStream_t stream) {
-  static int configured_device = -1;   // attribute is per device; re-set if the device changes
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<N, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<N>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  const cudaError_t e = set_smem_limit_once(mla_decode_kernel<N, T>, Cfg<N>::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(mla_decode_kernel<N, T>, grid, dim3(Cfg<N>::kThreads), Cfg<N>::kSmemBytes, stream, tm_k, tm_q, a);
 }
 

@@ -7,7 +7,24 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace mla {
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per device and process.
+// `done` holds one bit per device (0..63) that has been configured; concurrent first calls may both
+// set the attribute, which is idempotent.
+template <typename Kernel>
+inline cudaError_t set_smem_limit_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launch with programmatic stream serialization: the kernel may begin (prologue up to its
 // pdl_wait()) while the previous kernel of the stream is still running.
@@ -28,7 +45,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 struct DecodeArgs {
-  const uint8_t* k_cache;       // [num_pages, 64, h_kv, 576] bf16 (bytes, for L2 prefetch)
+  const uint8_t* k_cache;       // [num_pages, 64, h_kv, 576] bf16 or fp16 (read through the tensor maps)
   const int32_t* block_table;   // [batch, max_pages]
   const int32_t* seqlens;       // [batch]
   const int32_t* tile_md;       // [num_parts, 8]

@@ -609,15 +609,9 @@ int decode_pair_smem_bytes() { return kSmemBytes; }
 
 template <int T>
 static cudaError_t launch_pair_t(const PairMaps& maps, const DecodeArgs& a, int row_blocks, cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_pair_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  const cudaError_t e = set_smem_limit_once(mla_decode_pair_kernel<T>, kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   const int pairs = (row_blocks + 1) / 2;
   const dim3 grid(2 * pairs, a.h_kv, a.num_parts);
   return launch_pdl(mla_decode_pair_kernel<T>, grid, dim3(kThreads), kSmemBytes, stream, maps, a);

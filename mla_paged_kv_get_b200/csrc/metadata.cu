@@ -247,16 +247,11 @@ int metadata_max_parts() { return kMaxParts; }
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,
                             int32_t* num_splits, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(batch) * sizeof(long long) + (2 * batch + 1) * sizeof(int);
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    const int max_smem = kMaxBatch * static_cast<int>(sizeof(long long)) +
-                         (2 * kMaxBatch + 1) * static_cast<int>(sizeof(int));
-    cudaError_t e = cudaFuncSetAttribute(mla_metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  constexpr int kMaxSmem = kMaxBatch * static_cast<int>(sizeof(long long)) +
+                           (2 * kMaxBatch + 1) * static_cast<int>(sizeof(int));
+  static std::atomic<uint64_t> configured{0};
+  const cudaError_t e = set_smem_limit_once(mla_metadata_kernel, kMaxSmem, configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(mla_metadata_kernel, dim3(1), dim3(kThreads), smem, stream, seqlens, batch, num_parts, tile_md,
                     num_splits);
 }
