@@ -63,3 +63,20 @@ def test_decode_rejects_bad_arguments_without_a_gpu(lib):
     rc = lib.mla_decode_paged(None, None, 1, None, 1, None, 1, 1, 16, 1, 576, 512, None, None, 1, 0,
                               ctypes.c_float(0.04), None, 0, None, None, None, None)
     assert rc == -1
+
+
+def test_traffic_records_name_existing_decode_sources():
+    """The stored ncu traffic is reported only while the decode kernels' sources hash to the recorded
+    value: every file in that hash must exist, and each record must name a hash of the same form."""
+    import json
+    import bench
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    csrc = os.path.join(root, "mla_paged_kv_get_b200", "csrc")
+    for name in bench.DECODE_SOURCES:
+        assert os.path.isfile(os.path.join(csrc, name)), name
+    sha = bench.source_sha()
+    assert re.fullmatch(r"[0-9a-f]{16}", sha)
+    for rec in ("decode_compute_bound_traffic.json", "decode_varlen_memory_bound_traffic.json"):
+        with open(os.path.join(root, "profiles", rec)) as f:
+            d = json.load(f)
+        assert re.fullmatch(r"[0-9a-f]{16}", d["kernel_source_sha"]) and d["dram_bytes_per_launch"] > 0
