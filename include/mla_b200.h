@@ -17,6 +17,16 @@
  *     no device memory and never synchronises the stream.
  *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = legacy default stream).
+ *   - Kernels are launched with programmatic stream serialization: each may
+ *     start its set-up while the previous kernel of the stream is finishing,
+ *     and waits for that kernel to complete before reading or writing any
+ *     buffer, so stream order is kept.  The metadata and decode kernels, and
+ *     the combine kernel (which the decode call launches last), let the next
+ *     kernel start early in the same way: a kernel of the caller's launched
+ *     after them with programmatic serialization must itself wait for its
+ *     predecessor (griddepcontrol.wait / cudaGridDependencySynchronize) before
+ *     reading `out`, `lse`, `tile_md` or `num_splits`; one launched normally
+ *     needs nothing.
  *   - Return value: MLA_OK or a negative MLA_ERR_* code; on error nothing is
  *     launched.  Errors detected on the device (bad page ids, sequence longer
  *     than its block-table row, a bounded wait that ran out) are written to
