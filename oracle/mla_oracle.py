@@ -18,7 +18,7 @@ release list "BF16, 分頁kvcache 塊大小64"):
 * the call returns ``(out, lse)`` (cnblogs §6.2: ``output, lse =
   flash_mla_with_kvcache(...)``).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent (this project's choices):
 
 * ``lse`` is the natural logarithm, shape ``[B, s_q, h_q]``.
 * causal: the ``s_q`` query tokens are the last ``s_q`` positions of the

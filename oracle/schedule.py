@@ -8,7 +8,7 @@ GPU in parallel (jsxs2.com "ä»€éº¼æ˜¯FlashMLA", Â§3.1 åˆ†å¡Šèª¿åº¦èˆ‡ä¸¦è¡Œè¨ˆç®
 the metadata call takes the per-sequence lengths plus ``s_q*h_q//h_kv`` and
 ``h_kv`` and returns ``tile_scheduler_metadata, num_splits`` (cnblogs
 "DeepSeek å¼€æºè®°-ç¬¬1å¤©-FlashMLA", Â§6.2 åŸºæœ¬ä½¿ç”¨).  The concrete rule below is
-this project's reading, stated in full in DESIGN.md ("Scheduler rule"):
+this project's reading of them:
 
 * rows per KV head ``R = s_q*h_q/h_kv`` are cut into row blocks of
   ``N = 16`` (R <= 16), ``32`` (R <= 32) or ``64`` rows; ``T = ceil(R/N)``;
