@@ -2,13 +2,20 @@
 
 A step is the whole hot path over one batch: the metadata kernel, the split-KV
 decode kernel and the combine kernel, launched through the C ABI on one
-stream.  The default workload is the compute-bound decode configuration
+stream.  The headline workload is the compute-bound decode configuration
 (64 sequences x 4096 tokens, h_q = 128, one shared 576-wide KV head, 64-token
 pages, shuffled page table); its 302 MB cache is larger than the 126 MB L2,
 so consecutive steps do not hit in L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference]
+
+Without ``--workload`` the line also carries ``workloads``: the same
+measurement (its own timed region of 200 steps) for the tiny, variable-length
+memory-bound, causal MTP and long-context configurations.  Per-kernel device
+times come from separate loops of 64 back-to-back launches of one kernel
+between two CUDA events, after the timed region, so they never perturb the
+step time and never rest on a handful of samples.
 
 ``--impl reference`` times the fp64 CPU oracle on this machine's cores on a
 bounded sample of the same workload (the pages ship no runnable code).  Under
@@ -284,18 +291,185 @@ def run_reference(args, world, rank):
     return 0
 
 
+# The benchmark spec's class of each large workload and its target fraction of the nominal B200 peaks:
+# compute-bound configurations against 2.25 PFLOP/s dense bf16, the memory-bound one against 8 TB/s.
+GATES = {
+    "compute_bound": ("tensor", 0.5),
+    "varlen_memory_bound": ("hbm", 0.7),
+    "mtp_causal": ("tensor", 0.5),
+    "long_context_split_kv": ("tensor", 0.5),
+}
+NOMINAL = {"tensor": (2250.0, "TFLOP/s"), "hbm": (8000.0, "GB/s")}
+KERNEL_SAMPLES = 64          # back-to-back launches per kernel in the per-kernel loops
+SIDE_STEPS = 200             # timed steps of each further workload in the default run
+
+
+class Path:
+    """One workload's device buffers and the three C-ABI launches of a decode step."""
+
+    def __init__(self, w, dev, stream, lib):
+        from mla_paged_kv_get_b200 import binding
+        self.w, self.lib, self.stream = w, lib, stream
+        self.q, self.k, self.bt, self.sl = (w.q.to(dev), w.k_cache.to(dev), w.block_table.to(dev),
+                                            w.seqlens.to(dev))
+        self.R, self.h_kv = w.rows_per_kv, w.h_kv
+        self.G = binding.num_parts(self.R, self.h_kv)
+        self.tile_md = torch.empty((self.G, 8), dtype=torch.int32, device=dev)
+        self.num_splits = torch.empty((w.batch + 1,), dtype=torch.int32, device=dev)
+        self.ws = torch.empty((binding.workspace_bytes(w.batch, self.R, self.h_kv, self.G),), dtype=torch.uint8,
+                              device=dev)
+        self.out = torch.empty((w.batch, w.s_q, w.h_q, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.h = binding._stream_handle(stream)
+        self.P = binding._ptr
+        self.binding = binding
+
+    def metadata(self):
+        w, P = self.w, self.P
+        return self.lib.mla_get_metadata(P(self.sl), w.batch, self.R, self.h_kv, 0, P(self.tile_md),
+                                         P(self.num_splits), None, self.h)
+
+    def decode(self, flags=0):
+        w, P = self.w, self.P
+        return self.lib.mla_decode_paged_ex(
+            P(self.q), P(self.k), self.k.shape[0], P(self.bt), self.bt.shape[1], P(self.sl), w.batch, w.s_q,
+            w.h_q, self.h_kv, 576, 512, P(self.tile_md), P(self.num_splits), self.G, int(w.causal), w.scale,
+            P(self.ws), self.ws.numel(), P(self.out), P(self.lse), P(self.status), flags, 0, self.h)
+
+    def combine(self):
+        w, P = self.w, self.P
+        return self.lib.mla_combine(P(self.num_splits), P(self.ws), self.ws.numel(), w.batch, w.s_q, w.h_q,
+                                    self.h_kv, self.G, P(self.out), P(self.lse), self.h)
+
+    def step(self):
+        """metadata + decode + combine: the public two-call API (mla_decode_paged launches the combine)."""
+        return self.metadata() | self.decode(0)
+
+    def check_status(self):
+        st = int(self.status.item())
+        assert st == 0, self.binding.status_string(st)
+
+    def busy(self, seconds: float):
+        """Untimed steps for about `seconds`, so the clocks sampled next are clocks under load."""
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(20):
+                self.step()
+            torch.cuda.synchronize()
+
+    def kernel_ms(self, n: int = KERNEL_SAMPLES) -> dict:
+        """Device time per launch of each kernel alone: n back-to-back launches of one kernel
+        between two events on the launching stream (no event between launches, so each launch
+        still overlaps its predecessor's tail through programmatic launch, as inside a step)."""
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        s = self.stream
+        ev[0].record(s)
+        for _ in range(n):
+            self.metadata()
+        ev[1].record(s)
+        for _ in range(n):
+            self.decode(2)     # decode kernel only; the partials stay in the workspace
+        ev[2].record(s)
+        for _ in range(n):
+            self.combine()
+        ev[3].record(s)
+        torch.cuda.synchronize()
+        self.step()            # leave complete results behind
+        torch.cuda.synchronize()
+        return {"metadata": ev[0].elapsed_time(ev[1]) / n, "decode": ev[1].elapsed_time(ev[2]) / n,
+                "combine": ev[2].elapsed_time(ev[3]) / n, "samples": n}
+
+
+def fractions(flops: int, nbytes: int, seconds: float, peaks) -> dict:
+    tf = flops / seconds / 1e12
+    gbs = nbytes / seconds / 1e9
+    return {"tflops": tf, "hbm_gbs": gbs,
+            "tensor_frac_of_2250": tf / 2250.0, "hbm_frac_of_8000": gbs / 8000.0,
+            "tensor_frac_of_measured": tf / float(peaks["bf16_tflops"]),
+            "hbm_frac_of_measured": gbs / float(peaks["hbm_gbs"])}
+
+
+def gate(name: str, flops: int, nbytes: int, step_ms: float, decode_ms: float):
+    """The benchmark spec's gate for this workload: its class, target and the fraction of the nominal
+    peak reached by the whole step and by the decode kernel alone."""
+    if name not in GATES:
+        return {"class": "parity only (latency)", "step_us": step_ms * 1e3}
+    cls, target = GATES[name]
+    peak, unit = NOMINAL[cls]
+    work = flops / 1e12 if cls == "tensor" else nbytes / 1e9
+    f_step = work / (step_ms * 1e-3) / peak
+    f_dec = work / (decode_ms * 1e-3) / peak
+    return {"class": cls, "nominal_peak": peak, "unit": unit, "target_frac": target,
+            "frac_step": f_step, "frac_decode_kernel": f_dec, "met": f_step >= target,
+            "target_step_us": work / (target * peak) * 1e6}
+
+
+def measure(path, steps: int, warmup: int, world: int, dev, peaks) -> dict:
+    """Warm-up, then exactly `steps` timed steps between a barrier and a synchronize on both
+    sides, the per-kernel loops and the clocks sampled over both."""
+    w = path.w
+    for _ in range(warmup):
+        assert path.step() == 0
+    torch.cuda.synchronize(dev)
+    path.check_status()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index or 0)
+    with sampler:
+        path.busy(0.3)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(path.stream)
+        for _ in range(steps):
+            path.step()
+        stop.record(path.stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        km = path.kernel_ms()
+    path.check_status()
+    ms_step = max_over_ranks(start.elapsed_time(stop) / steps, world, dev)
+    decode_ms = max_over_ranks(km["decode"], world, dev)
+    combine_ms = max_over_ranks(km["combine"], world, dev)
+    metadata_ms = max_over_ranks(km["metadata"], world, dev)
+    flops, nbytes = algorithmic_work(w)
+    return {"w": w, "steps": steps, "ms_per_step": ms_step, "decode_ms": decode_ms, "combine_ms": combine_ms,
+            "metadata_ms": metadata_ms, "kernel_samples": km["samples"], "flops": flops, "bytes": nbytes,
+            "clocks": sampler.summary()}
+
+
+def workload_entry(m: dict, peaks) -> dict:
+    w = m["w"]
+    return {
+        "gate": gate(w.name, m["flops"], m["bytes"], m["ms_per_step"], m["decode_ms"]),
+        "ms_per_step": m["ms_per_step"], "steps": m["steps"],
+        "decode_us": m["decode_ms"] * 1e3, "combine_us": m["combine_ms"] * 1e3,
+        "metadata_us": m["metadata_ms"] * 1e3, "kernel_samples": m["kernel_samples"],
+        "algorithmic_flops": m["flops"], "algorithmic_bytes": m["bytes"],
+        "step": fractions(m["flops"], m["bytes"], m["ms_per_step"] * 1e-3, peaks),
+        "decode_kernel": fractions(m["flops"], m["bytes"], m["decode_ms"] * 1e-3, peaks),
+        "launch_ms_le_step": m["decode_ms"] <= m["ms_per_step"],
+        "config": {k: v for k, v in w.describe().items() if k != "workload"},
+        "clocks": m["clocks"],
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help="time this workload only (default: compute_bound as the headline, plus a "
+                         "'workloads' entry for every other configuration)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-torch-baseline", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    only = args.workload is not None
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD
 
     world, rank, local = dist_setup()
     if args.impl == "reference":
@@ -306,95 +480,36 @@ def main(argv=None):
         return rc
 
     from mla_paged_kv_get_b200 import binding
-    binding.load_library()
+    lib = binding.load_library()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
 
-    idx = WORKLOADS[args.workload]
-    w = inputs.config(idx)
-    flops, nbytes = algorithmic_work(w)
-    q, k, bt, sl = (w.q.to(dev), w.k_cache.to(dev), w.block_table.to(dev), w.seqlens.to(dev))
-    R, h_kv = w.rows_per_kv, w.h_kv
-    G = binding.num_parts(R, h_kv)
-    tile_md = torch.empty((G, 8), dtype=torch.int32, device=dev)
-    num_splits = torch.empty((w.batch + 1,), dtype=torch.int32, device=dev)
-    ws = torch.empty((binding.workspace_bytes(w.batch, R, h_kv, G),), dtype=torch.uint8, device=dev)
-    out = torch.empty((w.batch, w.s_q, w.h_q, 512), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    lib = binding.load_library()
-    h = binding._stream_handle(stream)
-    P = binding._ptr
-
-    def step():
-        rc = lib.mla_get_metadata(P(sl), w.batch, R, h_kv, 0, P(tile_md), P(num_splits), None, h)
-        rc |= lib.mla_decode_paged(P(q), P(k), k.shape[0], P(bt), bt.shape[1], P(sl), w.batch, w.s_q, w.h_q,
-                                   h_kv, 576, 512, P(tile_md), P(num_splits), G, int(w.causal),
-                                   w.scale, P(ws), ws.numel(), P(out), P(lse), P(status), h)
-        return rc
-
-    # events between the launches give per-kernel device time inside the timed region
-    def step_with_events(ev):
-        lib.mla_get_metadata(P(sl), w.batch, R, h_kv, 0, P(tile_md), P(num_splits), None, h)
-        ev[0].record(stream)
-        lib.mla_decode_paged_ex(P(q), P(k), k.shape[0], P(bt), bt.shape[1], P(sl), w.batch, w.s_q, w.h_q,
-                                h_kv, 576, 512, P(tile_md), P(num_splits), G, int(w.causal),
-                                w.scale, P(ws), ws.numel(), P(out), P(lse), P(status), 2, 0, h)
-        ev[1].record(stream)
-        lib.mla_combine(P(num_splits), P(ws), ws.numel(), w.batch, w.s_q, w.h_q, h_kv, G, P(out), P(lse), h)
-        ev[2].record(stream)
-
-    for _ in range(args.warmup):
-        assert step() == 0
-    torch.cuda.synchronize(dev)
-    assert int(status.item()) == 0, binding.status_string(int(status.item()))
-
-    # ---- timed region: K steps, barrier + sync on both sides.  Every EV_EVERY-th step carries
-    # events around the decode and combine launches (on the launching stream).  An event between
-    # two launches breaks their programmatic-launch overlap, so the instrumented steps are slower
-    # than the rest: they are kept few (500 steps -> 32 samples of each kernel).
-    EV_EVERY = 16
-    n_ev = min((args.steps + EV_EVERY - 1) // EV_EVERY, 512)
-    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_ev)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with sampler:
-        start.record(stream)
-        for i in range(args.steps):
-            if i % EV_EVERY == 0 and i // EV_EVERY < n_ev:
-                step_with_events(evs[i // EV_EVERY])
-            else:
-                step()
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    ms_total = start.elapsed_time(stop)
-    ms_total_max = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total_max / args.steps
-    decode_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)    # decode kernel alone
-    combine_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    assert int(status.item()) == 0, binding.status_string(int(status.item()))
+    w = inputs.config(WORKLOADS[args.workload])
+    path = Path(w, dev, stream, lib)
+    m = measure(path, args.steps, args.warmup, world, dev, peaks)
+    ms_step, decode_ms, flops, nbytes = m["ms_per_step"], m["decode_ms"], m["flops"], m["bytes"]
+    # The decode kernel alone cannot take longer than the step that contains it.
+    assert decode_ms <= ms_step * 1.02, (decode_ms, ms_step)
 
     # ---- end to end through the public API with host buffers (pinned), H2D + D2H inside the region
     hq, hk, hbt, hsl = (w.q.pin_memory(), w.k_cache.pin_memory(), w.block_table.pin_memory(),
                         w.seqlens.pin_memory())
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    hout = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+    hlse = torch.empty(path.lse.shape, dtype=path.lse.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hbt, hsl))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
 
     def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        bt.copy_(hbt, non_blocking=True)
-        sl.copy_(hsl, non_blocking=True)
-        assert step() == 0
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+        path.q.copy_(hq, non_blocking=True)
+        path.k.copy_(hk, non_blocking=True)
+        path.bt.copy_(hbt, non_blocking=True)
+        path.sl.copy_(hsl, non_blocking=True)
+        assert path.step() == 0
+        hout.copy_(path.out, non_blocking=True)
+        hlse.copy_(path.lse, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -406,8 +521,8 @@ def main(argv=None):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    path.check_status()
 
-    peaks, peak_src = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
     tc_peak = float(peaks["bf16_tflops"])
     dec_s = decode_ms * 1e-3
@@ -419,22 +534,22 @@ def main(argv=None):
     traffic, traffic_sha = load_traffic(w.name)
     if traffic_sha is not None and traffic_sha != source_sha():
         traffic = None   # counters were taken on another version of the kernels
+    roof = {"gate": gate(w.name, flops, nbytes, ms_step, decode_ms)}
     if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak}
+        roof.update({"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak})
     else:
-        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved_tf / tc_peak}
+        roof.update({"bound": "tensor", "achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": achieved_tf / tc_peak})
     roof.update({"traffic": traffic, "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
                  if peak_src == "measured" else "fallback",
-                 "kernel": ("mla_decode_pair_kernel" if R > 64 else "mla_decode_kernel")
-                 + f" (CUDA events around its launch on every {EV_EVERY}th timed step)",
-                 "combine_ms": combine_ms,
+                 "kernel": ("mla_decode_pair_kernel" if path.R > 64 else "mla_decode_kernel")
+                 + f" ({m['kernel_samples']} back-to-back decode-only launches between CUDA events, after the "
+                   "timed region)",
+                 "launch_ms": decode_ms, "combine_ms": m["combine_ms"], "metadata_ms": m["metadata_ms"],
+                 "launch_ms_le_step": decode_ms <= ms_step,
                  "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
-                 "launch_ms": decode_ms,
-                 "tensor_frac_of_measured": achieved_tf / tc_peak,
-                 "hbm_frac_of_measured": achieved_gbs / hbm_peak,
-                 "tensor_frac_of_2250": achieved_tf / 2250.0, "hbm_frac_of_8000": achieved_gbs / 8000.0})
+                 **{k: v for k, v in fractions(flops, nbytes, dec_s, peaks).items() if "frac" in k}})
 
     total_flops = flops * world
     line = {
@@ -454,10 +569,24 @@ def main(argv=None):
                 "ms_per_step": e2e_ms, "what": "pinned H2D of q, cache, page table, seqlens; "
                                              "metadata + decode + combine; D2H of out and lse"},
         "gpu_launches": 3 * args.steps,
-        "clocks": sampler.summary(),
+        "clocks": m["clocks"],
     }
+    del path
+    if world == 1 and not only:
+        # every other configuration, each in its own timed region of SIDE_STEPS steps
+        side = {}
+        for name in sorted(WORKLOADS, key=WORKLOADS.get):
+            if name == w.name:
+                continue
+            wl = inputs.config(WORKLOADS[name])
+            p = Path(wl, dev, stream, lib)
+            side[name] = workload_entry(measure(p, SIDE_STEPS, args.warmup, world, dev, peaks), peaks)
+            del p, wl
+            torch.cuda.empty_cache()
+        line["workloads"] = side
     if rank == 0 and world == 1 and not args.no_torch_baseline:
-        line["torch_baseline"] = torch_native_timing(w, q, k, bt, sl, flops)
+        line["torch_baseline"] = torch_native_timing(w, w.q.to(dev), w.k_cache.to(dev), w.block_table.to(dev),
+                                                     w.seqlens.to(dev), flops)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_timing(w)
     if rank == 0:

@@ -16,7 +16,8 @@
  *     must stay valid until the stream work completes.  The library allocates
  *     no device memory and never synchronises the stream.
  *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
- *     NULL = legacy default stream).
+ *     NULL = legacy default stream), which must belong to the current device:
+ *     kernels are launched on the current device.
  *   - Kernels are launched with programmatic stream serialization: each may
  *     start its set-up while the previous kernel of the stream is finishing,
  *     and waits for that kernel to complete before reading or writing any
@@ -126,8 +127,9 @@ size_t mla_workspace_bytes(int batch, int rows_per_kv, int h_kv, int dv, int num
  *   lse_d           fp32 [batch, s_q, h_q]; natural log; -inf for rows that
  *                   see no key (their out row is 0)
  *   status_d        optional int32 device word (see conventions)
- * Launches the decode kernel and, if any sequence is split or empty, the
- * combine kernel, both on `stream`.
+ * Launches the decode kernel and then the combine kernel, both on `stream`;
+ * the combine merges the rows of split sequences and zero-fills empty ones
+ * (its blocks for sequences the decode kernel finished return at once).
  */
 int mla_decode_paged(const void* q_d, const void* k_cache_d, int num_pages,
                      const int32_t* block_table_d, int max_pages_per_seq,
@@ -210,8 +212,14 @@ int mla_combine_typed(int dtype, const int32_t* num_splits_d, const void* worksp
  *   - Returns MLA_ERR_WORKSPACE if the shape needs more than
  *     MLA_NOALLOC_SCRATCH_BYTES (mla_workspace_bytes(...) larger than it).
  *   - The first call on a device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call outside any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and caches it together
+ *     with the unique id of the device's current context; a later call made
+ *     in another context of that device (for example after cudaDeviceReset
+ *     destroyed the old one) looks it up again.  Make the first call on a
+ *     device, and the first call after such a reset, outside any stream
+ *     capture.
+ *   - `stream` must belong to the current device (as for every call of this
+ *     library): the scratch array used is the current device's.
  *   - All calls share the one scratch array and it keeps the previous call's
  *     contents; nothing in it needs to start at zero (every partial is written
  *     before it is read).  Calls that overlap on the GPU (other streams, other

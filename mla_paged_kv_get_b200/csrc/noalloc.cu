@@ -1,6 +1,7 @@
 // noalloc.cu — mla_decode_paged_noalloc: the decode entry point for callers
 // that cannot allocate device memory.  The split partials live in a static
 // device array owned by the library instead of a caller-supplied workspace.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -16,20 +17,57 @@ __device__ __align__(256) unsigned char g_mla_noalloc_scratch[MLA_NOALLOC_SCRATC
 
 constexpr int kMaxDevices = 64;
 
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 = none yet).  Ids are
+// never reused within a process, so a context destroyed and re-created (for
+// example by cudaDeviceReset) gets a new one, unlike its handle, which may be.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  return ctx == nullptr || get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context of the current
+// device.  Looked up once per device (cudaGetSymbolAddress with that device
+// current) and again only when the device's context has changed since.
 int scratch_address(void** out) {
-  static void* addr[kMaxDevices] = {};
+  struct Entry {
+    void* addr;
+    unsigned long long ctx_id;
+  };
+  static Entry cache[kMaxDevices] = {};
   static std::mutex mu;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  unsigned long long ctx_id = 0;
+  if (!current_context_id(&ctx_id)) return MLA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (cache[dev].addr == nullptr || ctx_id == 0 || cache[dev].ctx_id != ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_mla_noalloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
-    addr[dev] = p;
+    // the lookup makes the device's primary context current if no context was
+    if (!current_context_id(&ctx_id) || ctx_id == 0) return MLA_ERR_CUDA;
+    cache[dev] = Entry{p, ctx_id};
   }
-  *out = addr[dev];
+  *out = cache[dev].addr;
   return MLA_OK;
 }
 

@@ -114,12 +114,16 @@ def decode_dense(q, k_cache, block_table, seqlens, h_kv: int, causal: bool, scal
     return out, lse
 
 
-def attention_weights(q_row, K: np.ndarray, scale: float) -> np.ndarray:
-    """Softmax weights ``exp(x_j - lse)`` of one query row over keys ``K``."""
-    x = scale * (as_f64(q_row) @ as_f64(K).T)
-    m = x.max()
+def attention_weights(q_rows, K: np.ndarray, scale: float) -> np.ndarray:
+    """Softmax weights ``exp(x_j - lse)`` of query rows over keys ``K``.
+
+    ``q_rows`` is one row ``[576]`` (result ``[n]``) or several ``[r, 576]``
+    (result ``[r, n]``, one distribution per row).
+    """
+    x = scale * (as_f64(q_rows) @ as_f64(K).T)
+    m = x.max(axis=-1, keepdims=True)
     e = np.exp(x - m)
-    return e / e.sum()
+    return e / e.sum(axis=-1, keepdims=True)
 
 
 def merge_partials(lse_parts, o_parts):

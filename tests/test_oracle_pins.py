@@ -105,6 +105,15 @@ def test_weights_are_a_distribution():
         p = mo.attention_weights(q[0, 0, h], K, w.scale)
         assert p.min() >= 0.0
         assert abs(p.sum() - 1.0) < 1e-12
+    # a block of rows gives one distribution per row, each equal to its single-row form
+    pb = mo.attention_weights(q[0, 0], K, w.scale)
+    assert pb.shape == (16, 257)
+    assert np.all(np.abs(pb.sum(axis=1) - 1.0) < 1e-12)
+    for h in range(16):
+        assert np.array_equal(pb[h], mo.attention_weights(q[0, 0, h], K, w.scale))
+    # closed forms: a zero query weighs every key 1/n; a single key weighs 1
+    assert np.allclose(mo.attention_weights(np.zeros((3, 576)), K, w.scale), 1.0 / 257, rtol=0, atol=1e-15)
+    assert mo.attention_weights(q[0, 0, :2], K[:1], w.scale).tolist() == [[1.0], [1.0]]
 
 
 def test_page_permutation_is_bit_identical():
