@@ -231,10 +231,11 @@ int mla_decode_paged_typed(int dtype, const void* q_d, const void* k_cache_d, in
     mla::PairMaps maps;
     if (!page_map(&maps.k, 3)) return MLA_ERR_CUDA;
     for (int rank = 0; rank < 2; ++rank) {
-      // dv quarter of rank r: columns 256 h + 128 r + 64 sub + c -> (64 cols, tokens, 2 sub, 2 halves, heads)
+      // dv quarter of rank r: columns 256 h + 128 r + 64 sub + c -> (64 cols, tokens, 2 sub, 2 halves, heads);
+      // a box is one dv half of one page: 64 tokens x 128 columns (16 KB)
       const cuuint64_t dims[5] = {64, tokens, 2, 2, static_cast<cuuint64_t>(h_kv)};
       const cuuint64_t strides[4] = {token_bytes, 128, 512, MLA_HEAD_DIM * 2ull};
-      const cuuint32_t box[5] = {64, 64, 2, 2, 1};
+      const cuuint32_t box[5] = {64, 64, 2, 1, 1};
       const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
       void* base = static_cast<char*>(const_cast<void*>(k_cache_d)) + 256 * rank;
       if (encode(&maps.v[rank], tmap_type, 5, base, dims, strides, box, estr,

@@ -68,7 +68,7 @@ cudaError_t launch_decode(int rows_per_block, int dtype, const CUtensorMap& tm_k
                           const DecodeArgs& a, int row_blocks, cudaStream_t stream);
 
 // Tensor maps of the pair kernel: the score product's page chunks (24 KB boxes),
-// each CTA rank's dv quarter of a page (32 KB boxes) and the 64 Q rows (72 KB).
+// each CTA rank's dv quarter of one dv half of a page (16 KB boxes) and the 64 Q rows (72 KB).
 struct PairMaps {
   CUtensorMap k;
   CUtensorMap v[2];
