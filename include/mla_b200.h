@@ -96,6 +96,12 @@ int mla_num_parts(int rows_per_kv, int h_kv, int num_sms);
  *   num_parts_out    host int*, out: G (may be NULL)
  * One single-CTA kernel; integer arithmetic only (bit-exact, deterministic).
  * Limits: batch <= 8192 and G <= 4096 (MLA_ERR_INVALID_ARG otherwise).
+ * The kernel reads cache_seqlens_d and computes the table before it waits for
+ * the previous kernel of the stream (it waits only before writing its
+ * outputs), so a kernel of the caller's that writes cache_seqlens_d right
+ * before this call must not let its dependents launch early
+ * (griddepcontrol.launch_dependents) before those writes.  Kernels launched
+ * without programmatic launch and copies need nothing: the stream orders them.
  */
 int mla_get_metadata(const int32_t* cache_seqlens_d, int batch, int rows_per_kv, int h_kv,
                      int num_sms, int32_t* tile_md_d, int32_t* num_splits_d,
@@ -116,7 +122,8 @@ size_t mla_workspace_bytes(int batch, int rows_per_kv, int h_kv, int dv, int num
  *   k_cache_d       bf16 [num_pages, 64, h_kv, d]          (16-byte aligned)
  *   block_table_d   int32 [batch, max_pages_per_seq]; entries for pages at
  *                   or beyond ceil(L_b/64) are never read
- *   cache_seqlens_d int32 [batch]; L_b <= 64 * max_pages_per_seq required
+ *   cache_seqlens_d int32 [batch]; L_b <= 64 * max_pages_per_seq required;
+ *                   batch <= 8192 (the limit of mla_get_metadata)
  *   d, dv           must be 576 and 512
  *   tile_md_d, num_splits_d, num_parts: exactly as produced by
  *                   mla_get_metadata for the same seqlens, rows_per_kv, h_kv

@@ -141,7 +141,7 @@ int mla_decode_paged_typed(int dtype, const void* q_d, const void* k_cache_d, in
       tile_md_d == nullptr || num_splits_d == nullptr || out_d == nullptr || lse_d == nullptr)
     return MLA_ERR_INVALID_ARG;
   if (d != MLA_HEAD_DIM || dv != MLA_VALUE_DIM) return MLA_ERR_UNSUPPORTED;
-  if (batch < 1 || batch > 65535 || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || num_pages < 1 ||
+  if (batch < 1 || batch > mla::metadata_max_batch() || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || num_pages < 1 ||
       num_pages > (1 << 24) || max_pages_per_seq < 1 || max_pages_per_seq > (1 << 24) || num_parts < 1 ||
       num_parts > 65535)
     return MLA_ERR_INVALID_ARG;
@@ -252,7 +252,7 @@ int mla_decode_paged_typed(int dtype, const void* q_d, const void* k_cache_d, in
   }
   if (le != cudaSuccess) return MLA_ERR_CUDA;
   if (debug_flags & 2) return MLA_OK;
-  if (mla::launch_combine(dtype, num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, s) !=
+  if (mla::launch_combine(dtype, num_splits_d, a.o_part, a.lse_part, a.out, lse_d, batch, s_q, h_q, h_kv, R, dev.sms, s) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;
@@ -264,7 +264,8 @@ int mla_combine_typed(int dtype, const int32_t* num_splits_d, const void* worksp
   if (dtype != MLA_DTYPE_BF16 && dtype != MLA_DTYPE_FP16) return MLA_ERR_INVALID_ARG;
   if (num_splits_d == nullptr || workspace_d == nullptr || out_d == nullptr || lse_d == nullptr)
     return MLA_ERR_INVALID_ARG;
-  if (batch < 1 || batch > 65535 || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 || num_parts < 1)
+  if (batch < 1 || batch > mla::metadata_max_batch() || s_q < 1 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0 ||
+      num_parts < 1)
     return MLA_ERR_INVALID_ARG;
   if (!aligned(out_d, 16) || !aligned(workspace_d, 256)) return MLA_ERR_INVALID_ARG;
   const int R = static_cast<int>(static_cast<long long>(s_q) * h_q / h_kv);
@@ -272,7 +273,10 @@ int mla_combine_typed(int dtype, const int32_t* num_splits_d, const void* worksp
   const size_t max_pieces = static_cast<size_t>(batch) + num_parts;
   const float* o_part = static_cast<const float*>(workspace_d);
   const float* lse_part = o_part + max_pieces * h_kv * R * MLA_VALUE_DIM;
-  if (mla::launch_combine(dtype, num_splits_d, o_part, lse_part, out_d, lse_d, batch, s_q, h_q, h_kv, R,
+  DeviceInfo dev;
+  const int st = device_info(&dev);
+  if (st != MLA_OK) return st;
+  if (mla::launch_combine(dtype, num_splits_d, o_part, lse_part, out_d, lse_d, batch, s_q, h_q, h_kv, R, dev.sms,
                           static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;

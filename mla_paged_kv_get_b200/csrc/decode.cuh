@@ -80,7 +80,7 @@ cudaError_t launch_decode_pair(int dtype, const PairMaps& maps, const DecodeArgs
                                cudaStream_t stream);
 
 cudaError_t launch_combine(int dtype, const int32_t* num_splits, const float* o_part, const float* lse_part,
-                           void* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R,
+                           void* out, float* lse, int batch, int s_q, int h_q, int h_kv, int R, int num_sms,
                            cudaStream_t stream);
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* tile_md,

@@ -84,8 +84,9 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   // prologue now; it reads tile_md and num_splits only after this grid has completed.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // This grid may itself start before the previous kernel of the stream has finished (the combine
-  // of an earlier step still reads num_splits): wait for it before reading or writing anything.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // of an earlier step still reads num_splits).  Everything up to the first write of an output
+  // reads only the lengths, which no kernel of this library writes, so it overlaps that kernel;
+  // griddepcontrol.wait comes just before the outputs are written.
   extern __shared__ long long smem_ll[];
   long long* p_incl = smem_ll;                                        // [batch]  P_{b+1}
   int* n_s = reinterpret_cast<int*>(p_incl + batch);                  // [batch]  pages
@@ -205,16 +206,16 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_part
   long long total_pieces;
   long long run_p = block_exclusive_scan(my_pieces, warp_buf, &total_pieces);
   for (int b = b0; b < b1; ++b) {
-    num_splits[b] = static_cast<int32_t>(run_p);
     ns_s[b] = static_cast<int>(run_p);
     const int nb = n_s[b];
     if (nb > 0) run_p += part_of(first_unit(b) + nb - 1) - part_of(first_unit(b)) + 1;
   }
-  if (tid == 0) {
-    num_splits[batch] = static_cast<int32_t>(total_pieces);
-    ns_s[batch] = static_cast<int>(total_pieces);
-  }
+  if (tid == 0) ns_s[batch] = static_cast<int>(total_pieces);
   __syncthreads();
+
+  // ---- outputs, once the previous kernel of the stream has finished with them
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int b = tid; b <= batch; b += kThreads) num_splits[b] = static_cast<int32_t>(ns_s[b]);
 
   // ---- parts.  Pieces are numbered part by part, which along the cost line is also sequence by
   // sequence, so the pieces before the part that begins at `be` are those of the sequences before
