@@ -291,8 +291,9 @@ def run_reference(args, world, rank):
     return 0
 
 
-# The benchmark spec's class of each large workload and its target fraction of the nominal B200 peaks:
-# compute-bound configurations against 2.25 PFLOP/s dense bf16, the memory-bound one against 8 TB/s.
+# The speed target of each large workload: its class and the fraction of the nominal B200 peak it is
+# meant to reach, compute-bound configurations against 2.25 PFLOP/s dense bf16, the memory-bound one
+# against 8 TB/s.
 GATES = {
     "compute_bound": ("tensor", 0.5),
     "varlen_memory_bound": ("hbm", 0.7),
@@ -391,8 +392,8 @@ def fractions(flops: int, nbytes: int, seconds: float, peaks) -> dict:
 
 
 def gate(name: str, flops: int, nbytes: int, step_ms: float, decode_ms: float):
-    """The benchmark spec's gate for this workload: its class, target and the fraction of the nominal
-    peak reached by the whole step and by the decode kernel alone."""
+    """The speed target of this workload: its class, the target fraction and the fraction of the
+    nominal peak reached by the whole step and by the decode kernel alone."""
     if name not in GATES:
         return {"class": "parity only (latency)", "step_us": step_ms * 1e3}
     cls, target = GATES[name]
