@@ -260,7 +260,7 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
   const uint32_t p_addr = smem_addr(ps);
 
   uint32_t ridx = 0;   // loads of this issuer's ring consumed so far
-  int tg = 0, qloads = 0, seg_i = 0;
+  int tg = 0, qloads = 0, seg_i = 0;   // seg_i: segments with tiles issued so far
   bool alive = true;
   SegIter it;
   it.init(md);
@@ -268,11 +268,7 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
 
   while (alive && it.next(a, s)) {
     const int tg0 = tg;
-    if (s.ntiles == 0) {
-      if (pv_role && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) { alive = false; break; }
-      ++seg_i;
-      continue;
-    }
+    if (s.ntiles == 0) continue;   // nothing to issue; its epilogue does not touch O in TMEM
     if (!pv_role) {
       if (!wait_phase_lean(&ct.q_full, qloads & 1, ctl)) { alive = false; break; }
       ++qloads;
@@ -309,6 +305,8 @@ __device__ void mma_role(const DecodeArgs& a, Ctrl& ct, uint8_t* slots, uint8_t*
     auto do_pv = [&](int t) -> bool {
       if (!pv_role) return true;
       const int tgl = tg0 + t, pb = tgl & 1;
+      // O in TMEM is overwritten from the first value product of a segment on: wait until the softmax
+      // has read out the previous segment that had tiles (one o_free phase per such segment)
       if (t == 0 && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
       if (!wait_phase_lean(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
       tc_fence_after();
@@ -575,8 +573,12 @@ __device__ void softmax_role(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
         a.lse_part[(static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + r] = ct.lse_row[tid];
       }
     }
-    tc_fence_before();
-    mbar_arrive(&ct.o_free);
+    // O may be overwritten again: signalled only after segments that had tiles, the ones whose O came
+    // from TMEM, so the value issuer (which waits once per such segment) can never be lapped
+    if (s.ntiles > 0) {
+      tc_fence_before();
+      mbar_arrive(&ct.o_free);
+    }
   }
 }
 

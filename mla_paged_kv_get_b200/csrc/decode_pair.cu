@@ -244,17 +244,13 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
   const uint32_t idesc_pv = idesc_f32<T>(128, 256, false, true);    // A = P (K-major), B = V (MN-major)
   const uint32_t q_addr = smem_addr(qs), p_addr = smem_addr(ps), k_addr = smem_addr(ks), v_addr = smem_addr(vs);
   uint32_t vidx = 0;
-  int tg = 0, qloads = 0, seg_i = 0;
+  int tg = 0, qloads = 0, seg_i = 0;   // seg_i: segments with tiles issued so far
   SegIter it;
   it.init(md);
   Seg s;
   while (it.next(a, s)) {
     const int tg0 = tg;
-    if (s.ntiles == 0) {
-      if (kValue && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
-      ++seg_i;
-      continue;
-    }
+    if (s.ntiles == 0) continue;   // nothing to issue; its epilogue does not touch O in TMEM
     if constexpr (!kValue) {
       if (!wait_phase_lean(&ct.q_full, qloads & 1, ctl)) return false;
       ++qloads;
@@ -287,6 +283,8 @@ __device__ bool mma_issue(const DecodeArgs& a, Ctrl& ct, uint8_t* qs, uint8_t* p
 #pragma unroll 1
       for (int t = 0; t < s.ntiles; ++t) {
         const int tgl = tg0 + t, pb = tgl & 1;
+        // O in TMEM is overwritten from the first value product of a segment on: wait until the
+        // softmax has read out the previous segment that had tiles (one o_free phase per such segment)
         if (t == 0 && seg_i > 0 && !wait_phase_lean(&ct.o_free, (seg_i - 1) & 1, ctl)) return false;
         if (!wait_phase_lean(&ct.p_full[pb], (tgl >> 1) & 1, ctl)) return false;
         tc_fence_after();
@@ -513,9 +511,13 @@ __device__ void softmax_rows(const DecodeArgs& a, Ctrl& ct, uint8_t* ps, uint32_
       else
         a.lse_part[(static_cast<size_t>(s.piece) * a.h_kv + g) * a.R + rr] = lse;
     }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(leader_o_free);
+    // O may be overwritten again: signalled only after segments that had tiles, the ones whose O came
+    // from TMEM, so the value issuer (which waits once per such segment) can never be lapped
+    if (s.ntiles > 0) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_o_free);
+    }
   }
 }
 

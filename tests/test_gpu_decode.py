@@ -203,6 +203,42 @@ def test_sequence_longer_than_its_block_table_row(h_q, sms):
     compare(w, out, lse, o_ref, l_ref, batches=good, what=f"overlong h_q={h_q} sms={sms}")
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("h_q,sms", [(16, 2), (16, 148), (128, 2), (128, 148)])
+def test_runs_of_overlong_sequences(h_q, sms):
+    """Runs of over-long sequences between valid ones: each is a segment without tiles in the
+    part that holds it (with two SMs, one part holds them all, back to back).  Every launch
+    reports MLA_ERR_BAD_INPUT with zero rows and lse = -inf for them, and the valid sequences
+    match the oracle, bit for bit from launch to launch.  The value-product issuer counts the
+    softmax's O hand-offs; had it lost count over the empty segments, it would wait out its
+    limit and abort the part, and the valid sequences after the run would come out wrong."""
+    w = inputs.build(f"overlong_run{h_q}", [300, 100, 100, 100, 200, 100, 100, 500, 64], s_q=1, h_q=h_q,
+                     seed=13)
+    max_pages = w.block_table.shape[1]
+    bad_rows, good = [1, 2, 3, 5, 6], [0, 4, 7, 8]
+    lens = w.seqlens.clone()
+    lens[bad_rows] = 64 * max_pages + 5
+    q, k, bt, _ = to_gpu(w)
+    sl = lens.cuda()
+    md, ns = binding.get_metadata(sl, w.rows_per_kv, w.h_kv, num_sms=sms)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o_ref, l_ref = oracle(w, batches=good)
+    out0 = lse0 = None
+    for i in range(20):
+        status.zero_()
+        out, lse = binding.decode_paged(q, k, bt, sl, 512, md, ns, softmax_scale=w.scale, status=status,
+                                        timeout_ns=200_000_000)
+        torch.cuda.synchronize()
+        assert int(status.item()) == binding.MLA_ERR_BAD_INPUT, binding.status_string(int(status.item()))
+        assert torch.all(out[bad_rows].float() == 0) and torch.all(torch.isneginf(lse[bad_rows]))
+        if i == 0:
+            compare(w, out, lse, o_ref, l_ref, batches=good, what=f"overlong run h_q={h_q} sms={sms}")
+            out0, lse0 = out.clone(), lse.clone()
+        else:
+            assert torch.equal(out[good].view(torch.int16), out0[good].view(torch.int16))
+            assert torch.equal(lse[good].view(torch.int32), lse0[good].view(torch.int32))
+
+
 @pytest.mark.parametrize("rows", [16, 32, 64, 128])
 def test_repeated_launches_are_bit_identical(rows):
     """Hundreds of back-to-back launches on the varlen lengths of the memory-bound
